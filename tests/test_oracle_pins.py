@@ -1,0 +1,326 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+* Hadamard: scipy's Sylvester construction, H H^T = b I, the explicit (-1)^popcount(i&j) matrix,
+  and the involution H(Hx) = b x -- exact on small integers.
+* Transform: a float64 reference built from scipy's Hadamard matrix, within the fp32 rounding bound,
+  and absorption invariance X diag(1/s) H (W diag(s) H / b)^T = X W^T to 1e-5.
+* MXFP4: the hand-derived OCP MX v1.0 cases in tests/golden/ocp_mxfp4_cases.txt, a brute-force
+  nearest-grid search (a second, independent restatement written here), the defining property of
+  the shared exponent (block maximum lands in E2M1's top binade), and exact round trips of on-grid
+  values for every code and every reachable scale.
+* GEMM: an exact rational sum (fractions) on tiny shapes.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "ocp_mxfp4_cases.txt")
+GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _golden(kind):
+    out = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            if parts[0] == kind:
+                out.append(parts[1:])
+    return out
+
+
+# ---------------------------------------------------------------- Hadamard
+@pytest.mark.parametrize("b", [2, 4, 8, 16, 32, 64, 128])
+def test_fwht_matrix_is_sylvester(b):
+    cols = [oracle.fwht_f32(np.eye(b, dtype=np.float32)[j]) for j in range(b)]
+    H = np.stack(cols, axis=1).astype(np.float64)  # column j = H e_j
+    np.testing.assert_array_equal(H, scipy.linalg.hadamard(b).astype(np.float64))
+    np.testing.assert_array_equal(H @ H.T, b * np.eye(b))
+    explicit = np.array([[(-1) ** bin(i & j).count("1") for j in range(b)] for i in range(b)], np.float64)
+    np.testing.assert_array_equal(H, explicit)
+
+
+@pytest.mark.parametrize("b", [16, 32, 64, 128])
+def test_fwht_exact_on_small_integers_and_involution(b):
+    rng = np.random.default_rng(b)
+    explicit = np.array([[(-1) ** bin(i & j).count("1") for j in range(b)] for i in range(b)], np.float64)
+    for _ in range(20):
+        x = rng.integers(-1000, 1000, size=b).astype(np.float32)
+        y = oracle.fwht_f32(x)
+        np.testing.assert_array_equal(y.astype(np.float64), explicit @ x.astype(np.float64))
+        np.testing.assert_array_equal(oracle.fwht_f32(y).astype(np.float64), b * x.astype(np.float64))
+
+
+def _blockdiag_h(K, b):
+    H = scipy.linalg.hadamard(b).astype(np.float64)
+    return scipy.linalg.block_diag(*([H] * (K // b)))
+
+
+@pytest.mark.parametrize("b", [1, 16, 32, 64, 128])
+@pytest.mark.parametrize("absorb", [False, True])
+def test_transform_matches_float64_reference(b, absorb):
+    g = torch.Generator().manual_seed(7 + b)
+    K, rows = 256, 8
+    x = (torch.randn(rows, K, generator=g) * 3).to(torch.bfloat16)
+    m = torch.exp(torch.rand(K, generator=g) * 2.77 - 0.69).to(torch.float32)
+    y = oracle.transform_rows(x, m, b, absorb)
+    xd = x.to(torch.float64).numpy()
+    md = m.to(torch.float64).numpy()
+    Hb = _blockdiag_h(K, b) if b > 1 else np.eye(K)
+    ref = (xd * md) @ Hb
+    if absorb and b > 1:
+        ref = ref / b
+    absterm = np.abs(xd * md) @ np.abs(Hb)
+    if absorb and b > 1:
+        absterm = absterm / b
+    bound = (math.log2(b) + 2) * 2.0 ** -24 * absterm + 1e-30
+    assert np.all(np.abs(y.astype(np.float64) - ref) <= bound)
+
+
+@pytest.mark.parametrize("b", [16, 32, 64, 128])
+def test_absorption_invariance(b):
+    """X diag(1/s) H_b (W diag(s) H_b / b)^T equals X W^T to 1e-5 relative (unquantized)."""
+    g = torch.Generator().manual_seed(100 + b)
+    M, K, N = 12, 512, 24
+    X = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    X[:, :4] *= 50
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    s = torch.exp(torch.rand(K, generator=g) * 2.77 - 0.69).to(torch.float32)
+    inv_s = np.float32(1.0) / s.numpy()
+    xa = oracle.transform_rows(X, inv_s, b, absorb=False).astype(np.float64)
+    wa = oracle.transform_rows(W, s, b, absorb=True).astype(np.float64)
+    got = xa @ wa.T
+    ref = X.to(torch.float64).numpy() @ W.to(torch.float64).numpy().T
+    scale = np.abs(X.to(torch.float64).numpy()) @ np.abs(W.to(torch.float64).numpy()).T
+    assert np.max(np.abs(got - ref) / scale) < 1e-5
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-5
+
+
+def test_absorption_breaks_without_inverse_factor():
+    """The pin has teeth: dropping the 1/b factor (a plausible mistake) fails it by far."""
+    g = torch.Generator().manual_seed(5)
+    X = torch.randn(4, 64, generator=g).to(torch.bfloat16)
+    W = torch.randn(8, 64, generator=g).to(torch.bfloat16)
+    xa = oracle.transform_rows(X, None, 32, absorb=False).astype(np.float64)
+    wa_wrong = oracle.transform_rows(W, None, 32, absorb=False).astype(np.float64)
+    ref = X.double().numpy() @ W.double().numpy().T
+    assert np.linalg.norm(xa @ wa_wrong.T - ref) / np.linalg.norm(ref) > 1.0
+
+
+# ---------------------------------------------------------------- E2M1 / E8M0
+def brute_force_code(t: float) -> int:
+    """Nearest E2M1 magnitude by exhaustive search in exact rationals; a tie goes to the code with
+    an even mantissa bit (code bit 0); |t| > 6 clamps to 6; the sign bit follows the input's sign."""
+    sign = 8 if math.copysign(1.0, t) < 0 else 0
+    a = Fraction(abs(t)) if math.isfinite(t) else Fraction(10 ** 40)
+    best = None
+    for code, v in enumerate(GRID):
+        d = abs(a - Fraction(v))
+        if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
+            best = (d, code)
+    return sign | best[1]
+
+
+def test_e2m1_golden_cases():
+    cases = _golden("code")
+    assert len(cases) >= 20
+    for val, code, *_ in cases:
+        t = float(np.float32(float(val)))
+        assert oracle.e2m1_code(t) == int(code, 16), (val, code)
+        assert brute_force_code(t) == int(code, 16), (val, code)
+
+
+def test_e2m1_matches_brute_force_on_ties_and_random():
+    pts = []
+    for i in range(len(GRID) - 1):  # every midpoint and its fp32 neighbours
+        mid = np.float32((GRID[i] + GRID[i + 1]) / 2)
+        pts += [mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(10))]
+    pts += [np.float32(v) for v in GRID] + [np.float32(6.0001), np.float32(1e-45), np.float32(3e38)]
+    rng = np.random.default_rng(0)
+    pts += list(rng.uniform(0, 8, 4000).astype(np.float32))
+    pts += list((rng.standard_normal(2000) * 3).astype(np.float32))
+    for p in pts:
+        for t in (float(p), -float(p)):
+            assert oracle.e2m1_code(t) == brute_force_code(t), t
+
+
+def test_e8m0_golden_cases():
+    for amax, E, *_ in _golden("exp"):
+        assert oracle.e8m0_exponent(float(np.float32(float(amax)))) == int(E), amax
+
+
+def test_e8m0_puts_block_max_in_top_binade():
+    """Defining property of the shared exponent: amax / 2^(E-127) lies in [4, 8) whenever E is not
+    clamped, i.e. the largest element uses E2M1's top exponent (emax_elem = 2)."""
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        np.exp2(rng.uniform(-120, 125, 3000)),
+        np.exp2(np.arange(-124, 126)),                      # exact powers of two
+        np.nextafter(np.exp2(np.arange(-120, 126)).astype(np.float32), np.float32(0)),  # just below them
+    ]).astype(np.float32)
+    for a in vals:
+        E = oracle.e8m0_exponent(float(a))
+        r = Fraction(float(a)) / Fraction(2) ** (E - 127)
+        assert 4 <= r < 8, (a, E)
+
+
+def test_mxfp4_pack_golden():
+    for v0, v1, E, byte in _golden("pack"):
+        E = int(E)
+        y = np.zeros(32, np.float32)
+        y[0], y[1] = float(v0), float(v1)
+        y[31] = 4.0 * 2.0 ** (E - 127)
+        codes, sf = oracle.mxfp4_quantize(y)
+        assert int(sf[0, 0]) == E
+        assert int(codes[0, 0]) == int(byte, 16), (v0, v1, hex(codes[0, 0]))
+
+
+def test_mxfp4_round_trip_every_code_every_scale():
+    """Values already on the MXFP4 grid come back bit-exactly, for all 16 codes and every E8M0
+    value reachable from finite fp32 data (0..252)."""
+    codes16 = np.arange(16, dtype=np.uint8)
+    vals = np.array([oracle.e2m1_value(int(c)) for c in codes16])
+    assert list(vals[:8]) == GRID and list(-vals[8:]) == GRID
+    for E in range(0, 253):
+        y = np.zeros(32, np.float64)
+        y[:16] = vals
+        y[16:] = vals[::-1]
+        y = (y * 2.0 ** (E - 127)).astype(np.float32)
+        assert np.all(np.isfinite(y))
+        codes, sf = oracle.mxfp4_quantize(y)
+        assert int(sf[0, 0]) == E
+        expect = np.concatenate([codes16, codes16[::-1]])
+        got = np.empty(32, np.uint8)
+        got[0::2] = codes[0] & 15
+        got[1::2] = codes[0] >> 4
+        np.testing.assert_array_equal(got, expect)
+        back = oracle.dequant(codes, sf)[0]
+        np.testing.assert_array_equal(back, y.astype(np.float64))
+
+
+def test_mxfp4_quantize_matches_brute_force_rows():
+    rng = np.random.default_rng(3)
+    y = (rng.standard_normal((16, 128)) * np.exp2(rng.integers(-20, 20, (16, 1)))).astype(np.float32)
+    y[3] = 0
+    y[4, :32] = 1e-40
+    codes, sf = oracle.mxfp4_quantize(y)
+    for r in range(16):
+        for g in range(4):
+            blk = y[r, 32 * g:32 * g + 32]
+            amax = float(np.max(np.abs(blk)))
+            if amax == 0:
+                E = 0
+            else:
+                p = math.floor(math.log2(Fraction(amax))) if amax >= 2.0 ** -149 else -149
+                # exact floor(log2) by search (log2 of a Fraction is float; correct it exactly)
+                while Fraction(2) ** p > Fraction(amax):
+                    p -= 1
+                while Fraction(2) ** (p + 1) <= Fraction(amax):
+                    p += 1
+                E = min(max(p - 2 + 127, 0), 254)
+            assert sf[r, g] == E
+            for i in range(32):
+                t = float(Fraction(float(blk[i])) / Fraction(2) ** (E - 127))
+                c = (codes[r, (32 * g + i) // 2] >> (4 * (i & 1))) & 15
+                assert c == brute_force_code(t), (r, g, i)
+
+
+# ---------------------------------------------------------------- GEMM
+def test_linear_exact_rational_sum():
+    rng = np.random.default_rng(11)
+    for M, N, K in [(1, 1, 32), (3, 5, 64), (7, 4, 64)]:
+        Aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+        Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+        Asf = rng.integers(100, 150, (M, K // 32), dtype=np.uint8)
+        Wsf = rng.integers(100, 150, (N, K // 32), dtype=np.uint8)
+        Y, T = oracle.linear(Aq, Asf, Wq, Wsf)
+
+        def val(q, sf, r, k):
+            c = (q[r, k // 2] >> (4 * (k & 1))) & 15
+            mag = Fraction(GRID[c & 7])
+            return (-mag if c & 8 else mag) * Fraction(2) ** (int(sf[r, k // 32]) - 127)
+
+        for m in range(M):
+            for n in range(N):
+                terms = [val(Aq, Asf, m, k) * val(Wq, Wsf, n, k) for k in range(K)]
+                exact = sum(terms, Fraction(0))
+                tabs = sum((abs(t) for t in terms), Fraction(0))
+                assert abs(Fraction(Y[m, n]) - exact) <= Fraction(1, 10 ** 12) * tabs
+                assert abs(Fraction(T[m, n]) - tabs) <= Fraction(1, 10 ** 12) * tabs
+
+
+def test_linear_row_subset_and_grouped_reduce_to_dense():
+    rng = np.random.default_rng(12)
+    M, N, K, E = 20, 6, 128, 3
+    Aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    Asf = rng.integers(110, 140, (M, K // 32), dtype=np.uint8)
+    Wq = rng.integers(0, 256, (E, N, K // 2), dtype=np.uint8)
+    Wsf = rng.integers(110, 140, (E, N, K // 32), dtype=np.uint8)
+    off = np.array([0, 7, 7, 20], np.int32)  # expert 1 is empty
+    Yg, Tg = oracle.grouped_linear(Aq, Asf, off, Wq, Wsf)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        if hi == lo:
+            continue
+        Yd, Td = oracle.linear(Aq[lo:hi], Asf[lo:hi], Wq[e], Wsf[e])
+        np.testing.assert_array_equal(Yg[lo:hi], Yd)
+        np.testing.assert_array_equal(Tg[lo:hi], Td)
+    rows = [19, 0, 8]
+    Ys, _ = oracle.grouped_linear(Aq, Asf, off, Wq, Wsf, rows=rows)
+    np.testing.assert_array_equal(Ys, Yg[sorted(rows)])
+    Yd, _ = oracle.linear(Aq, Asf, Wq[2], Wsf[2], rows=[3, 9])
+    Yf, _ = oracle.linear(Aq, Asf, Wq[2], Wsf[2])
+    np.testing.assert_array_equal(Yd, Yf[[3, 9]])
+
+
+# ---------------------------------------------------------------- composed pipeline
+def test_prep_and_act_quant_compose_to_transform_then_quantize():
+    g = torch.Generator().manual_seed(21)
+    M, K, N, b = 5, 256, 7, 32
+    X = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    s = torch.exp(torch.rand(K, generator=g) * 2.77 - 0.69).to(torch.float32)
+    Wq, Wsf, inv_s = oracle.prep_weights(W, s, b)
+    np.testing.assert_array_equal(inv_s, np.float32(1.0) / s.numpy())
+    c2, s2 = oracle.mxfp4_quantize(oracle.transform_rows(W, s, b, absorb=True))
+    np.testing.assert_array_equal(Wq, c2)
+    np.testing.assert_array_equal(Wsf, s2)
+    Xq, Xsf = oracle.act_quant(X, inv_s, b)
+    c3, s3 = oracle.mxfp4_quantize(oracle.transform_rows(X, inv_s, b, absorb=False))
+    np.testing.assert_array_equal(Xq, c3)
+    np.testing.assert_array_equal(Xsf, s3)
+    # grouped act-quant reduces to the dense one per expert
+    inv2 = np.stack([inv_s, inv_s[::-1].copy()])
+    off = [0, 2, 5]
+    Gq, Gsf = oracle.act_quant(X, inv2, b, offsets=off)
+    for e in range(2):
+        q, sf = oracle.act_quant(X[off[e]:off[e + 1]], inv2[e], b)
+        np.testing.assert_array_equal(Gq[off[e]:off[e + 1]], q)
+        np.testing.assert_array_equal(Gsf[off[e]:off[e + 1]], sf)
+
+
+def test_quantized_layer_approximates_unquantized_product():
+    """End-to-end sanity: the W4A4 product stays close to X W^T (MXFP4 noise only). A random,
+    uncalibrated s spreads channel magnitudes 16x and costs accuracy; that is expected."""
+    g = torch.Generator().manual_seed(22)
+    M, K, N, b = 16, 512, 32, 32
+    X = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    X[:, [3, 100]] *= 50
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    s = torch.exp(torch.rand(K, generator=g) * 2.77 - 0.69).to(torch.float32)
+    ref = X.double().numpy() @ W.double().numpy().T
+    for scale, bound in ((None, 0.25), (s, 0.6)):
+        Wq, Wsf, inv_s = oracle.prep_weights(W, scale, b)
+        Xq, Xsf = oracle.act_quant(X, inv_s, b)
+        Y, _ = oracle.linear(Xq, Xsf, Wq, Wsf)
+        rel = np.linalg.norm(Y - ref) / np.linalg.norm(ref)
+        assert rel < bound, rel
