@@ -1,0 +1,186 @@
+/*
+ * macaq.h -- C ABI of libmacaq.so: the W4A4 / MXFP4 linear layer of MACaQ on NVIDIA B200 (sm_100a).
+ *
+ * The method. Page "Huawei's research lab in Switzerland open-sources the four-bit quantization tool
+ * MACaQ for running models locally" (aipolix.com, Persian), paragraph 2: at inference every layer's
+ * activations receive a per-channel scale and a small block-diagonal Hadamard transform, and the
+ * inverse is absorbed into the same layer's weights; paragraph 3: the target format is MXFP4 with
+ * 4-bit weights and activations (W4A4). Page "MACaQ quantizer from huawei-csl targets GGUF, vLLM and
+ * Diffusers models" (glonce.com), paragraph 5: the W4A4 dense and grouped matmuls. The MXFP4 rule is
+ * OCP Microscaling Formats (MX) v1.0: E2M1 elements, one E8M0 scale 2^(floor(log2 amax) - 2) per 32
+ * contiguous K elements, round-to-nearest-even, saturation at +-6.
+ *
+ * Concretely, with H_b the Sylvester Hadamard matrix of order b (entries +-1, natural order) applied
+ * to each aligned block of b input channels:
+ *     weights (offline):  W'  = MXFP4( W * diag(s) * H_b * (1/b) )
+ *     activations:        X'  = MXFP4( X * diag(1/s) * H_b )
+ *     output:             Y   = X' * W'^T   (fp32 accumulation, bf16 or fp32 result)
+ * so that Y approximates X * W^T (H_b * H_b^T = b * I). b = 1 means "no Hadamard" and a NULL scale
+ * means s = 1: together they give the plain-MXFP4 pipeline the overhead figure is measured against.
+ *
+ * Notation: M rows (tokens), K input channels, N output channels. All matrices are row-major.
+ *
+ * Data layouts (all buffers are device memory unless stated otherwise):
+ *   bf16 matrices        [rows, K], 2 bytes per element.
+ *   FP4 codes            [rows, K/2] bytes; element k of a row is nibble (k & 1) of byte k/2
+ *                        (even k in the low nibble); code = sign<<3 | E2M1 magnitude code.
+ *   scale factors (SF)   one E8M0 byte per 32 K-elements, stored in the tcgen05 block-scale tiling:
+ *                        rows are padded to a multiple of 128 and cut into 128 x 4 tiles (128 rows, 4
+ *                        scale columns = 128 K-elements); tiles are ordered row-tile-major, then by
+ *                        K-tile; inside a tile, row r and column c sit at byte
+ *                        (r % 32) * 16 + (r / 32) * 4 + c. Padding rows hold 0.
+ *                        Size: macaq_sf_bytes(rows, K).
+ *   grouped SF           the same tiling, but each expert's rows start on a fresh 128-row tile:
+ *                        expert e occupies row tiles [sum_{e'<e} ceil(M_e'/128), ...).
+ *                        Size bound: macaq_grouped_sf_bytes(total_rows, E, K).
+ *
+ * Conventions:
+ *   - The caller allocates and owns every buffer. The library never allocates device memory,
+ *     never frees it, and never synchronizes the device or the stream.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and returns a status. A launch failure returns MACAQ_ERR_CUDA (the cudaGetLastError code is
+ *     kept and can be read with macaq_last_cuda_error()). No exception crosses the ABI.
+ *   - Shape rules: K % 128 == 0 (whole 128 x 4 scale tiles); N % 128 == 0; M >= 0 (M == 0 is a
+ *     no-op); had_block in {1, 16, 32, 64, 128}. Every pointer argument must be 16-byte aligned.
+ *     Violations return MACAQ_ERR_SHAPE / MACAQ_ERR_ALIGNMENT / MACAQ_ERR_UNSUPPORTED /
+ *     MACAQ_ERR_INVALID_ARG before anything is launched.
+ *   - Device-side waits (pipeline barriers inside the GEMM) are bounded. A wait that runs out sets a
+ *     sticky device status word and the kernel returns without finishing; macaq_device_status()
+ *     reads that word (MACAQ_ERR_TIMEOUT) after the caller synchronizes.
+ *   - Calls are thread-safe; host-side tensor-map descriptors are cached under a mutex.
+ */
+#ifndef MACAQ_H
+#define MACAQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MACAQ_OK = 0,
+    MACAQ_ERR_INVALID_ARG = 1, /* NULL where a buffer is required, unknown enum value */
+    MACAQ_ERR_SHAPE = 2,       /* a dimension breaks the shape rules above */
+    MACAQ_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+    MACAQ_ERR_UNSUPPORTED = 4, /* had_block not supported, or the device is not sm_100 */
+    MACAQ_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
+    MACAQ_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out (see macaq_device_status) */
+    MACAQ_ERR_WORKSPACE = 7    /* workspace missing or smaller than macaq_workspace_bytes() */
+} macaq_status;
+
+typedef enum { MACAQ_OUT_BF16 = 0, MACAQ_OUT_F32 = 1 } macaq_out_dtype;
+
+/* How operand A of the GEMM is given: already quantized (codes + SF from macaq_act_quant), or as
+ * bf16 activations that the GEMM transforms and quantizes itself (the fused variant). */
+typedef enum { MACAQ_A_QUANTIZED = 0, MACAQ_A_BF16_FUSED = 1 } macaq_a_mode;
+
+/* A cudaStream_t, passed as a plain pointer so that this header needs no CUDA include. */
+typedef void *macaq_stream_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *macaq_status_str(int status);
+
+/* The cudaError_t of the most recent failing CUDA call made by this library on this thread. */
+int macaq_last_cuda_error(void);
+
+/* Bytes of the tiled scale-factor buffer for `rows` rows of K elements:
+ * ceil(rows / 128) * 128 * (K / 32). 0 for rows <= 0 or K not a multiple of 128. */
+size_t macaq_sf_bytes(int64_t rows, int64_t K);
+
+/* Upper bound of the grouped scale-factor buffer: (ceil(total_rows / 128) + E) * 128 * (K / 32).
+ * Every expert's rows start on a fresh 128-row tile, so at most E extra tiles are needed. */
+size_t macaq_grouped_sf_bytes(int64_t total_rows, int32_t E, int64_t K);
+
+/* Workspace bytes macaq_linear / macaq_grouped_linear need for these sizes (E = 0 for dense).
+ * 0 means no workspace is needed and `workspace` may be NULL. */
+size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E);
+
+/*
+ * Offline weight preparation (the absorbed inverse transform).
+ * Computes, per weight row and per aligned block of had_block channels, in fp32:
+ *     v = fl32(W[n,k] * s[k]);  v = v * H_b (fixed butterfly order h = 1, 2, ..., b/2);  v *= 1/b;
+ * then MXFP4 per 32 channels; also inv_s[k] = fl32(1 / s[k]) (IEEE division) for the activations.
+ *   W       device bf16 [N, K] (read)
+ *   s       device fp32 [K] per-channel scale, > 0 (read); NULL means s = 1 (then inv_s is untouched)
+ *   Wq      device u8 [N, K/2] (written)
+ *   Wsf     device u8, macaq_sf_bytes(N, K) bytes, tiled layout (written, padding rows zeroed)
+ *   inv_s   device fp32 [K] (written when s != NULL; may be NULL to skip)
+ * Source: the aipolix.com page, paragraph 2 (absorb the inverse into the same layer's weights).
+ */
+macaq_status macaq_prep_weights(const void *W, const float *s, int64_t N, int64_t K, int32_t had_block,
+                                uint8_t *Wq, uint8_t *Wsf, float *inv_s, macaq_stream_t stream);
+
+/*
+ * Online activation quantization: Xq/Xsf = MXFP4( X * diag(inv_s) * H_b ), in fp32 with the same
+ * fixed butterfly order, then OCP MX v1.0 quantization per 32 channels.
+ *   X              device bf16 [M, K] (read)
+ *   inv_s          device fp32 [K] (dense) or [E, K] (grouped); NULL means 1
+ *   group_offsets  NULL for a dense call; else device int32 [E + 1] (1 <= E <= 16384),
+ *                  non-decreasing, offsets[0] = 0,
+ *                  offsets[E] = M: rows [offsets[e], offsets[e+1]) belong to expert e and use
+ *                  inv_s + e*K. The values are read on the device; out-of-range offsets are clamped
+ *                  into [0, M] so no access leaves the buffers, but give undefined results.
+ *   Xq             device u8 [M, K/2] (written)
+ *   Xsf            device u8 (written): dense: macaq_sf_bytes(M, K) bytes; grouped: the per-expert
+ *                  padded tiling, at most macaq_grouped_sf_bytes(M, E, K) bytes. Padding rows get 0.
+ * Sources: aipolix.com page, paragraph 2 (per-channel scale and block Hadamard at inference) and
+ * paragraph 3 (MXFP4); glonce.com page, paragraph 5 (grouped matmul).
+ */
+macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64_t K, int32_t had_block,
+                             const int32_t *group_offsets, int32_t E, uint8_t *Xq, uint8_t *Xsf,
+                             macaq_stream_t stream);
+
+/*
+ * Dense W4A4 linear: Y[m, n] = sum_k dq(A[m, k]) * dq(W'[n, k]), fp32 accumulation on the tcgen05
+ * tensor cores (kind::mxf4 block-scaled MMA), written as bf16 (round-to-nearest-even) or fp32.
+ *   mode == MACAQ_A_QUANTIZED:  A = Xq device u8 [M, K/2], Asf = Xsf (tiled, macaq_sf_bytes(M, K)),
+ *                               inv_s and had_block are ignored.
+ *   mode == MACAQ_A_BF16_FUSED: A = X device bf16 [M, K], inv_s device fp32 [K] (NULL = 1), and the
+ *                               kernel applies scale, Hadamard and MXFP4 itself, bit-identical to
+ *                               macaq_act_quant; Asf is ignored.
+ *   Wq, Wsf    from macaq_prep_weights: u8 [N, K/2] and the tiled SF of N rows
+ *   Y          device [M, N], bf16 or fp32 per out_dtype (written)
+ *   workspace  device scratch of at least macaq_workspace_bytes(M, N, K, 0) bytes (NULL if 0)
+ * Source: glonce.com page, paragraph 5 (W4A4 dense matmul).
+ */
+macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M,
+                          int64_t N, int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf,
+                          void *Y, int32_t out_dtype, void *workspace, size_t ws_bytes,
+                          macaq_stream_t stream);
+
+/*
+ * Grouped (MoE) W4A4 linear: rows [offsets[e], offsets[e+1]) of A are multiplied by expert e's
+ * weights. A must already be quantized by macaq_act_quant in grouped form (mode must be
+ * MACAQ_A_QUANTIZED in this version; other modes return MACAQ_ERR_UNSUPPORTED).
+ *   A, Asf         Xq [total_rows, K/2] and the grouped tiled SF
+ *   group_offsets  device int32 [E + 1] (as for macaq_act_quant); 1 <= E <= 1024
+ *   Wq             device u8 [E, N, K/2];  Wsf device u8 [E, macaq_sf_bytes(N, K)]
+ *   Y              device [total_rows, N] (written; only rows of some expert are written)
+ *   workspace      device scratch of macaq_workspace_bytes(total_rows, N, K, E) bytes (NULL if 0)
+ * Source: glonce.com page, paragraph 5 (W4A4 grouped matmul).
+ */
+macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
+                                  const int32_t *group_offsets, int32_t E, int64_t total_rows, int64_t N,
+                                  int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf,
+                                  void *Y, int32_t out_dtype, void *workspace, size_t ws_bytes,
+                                  macaq_stream_t stream);
+
+/*
+ * Reads the sticky device status word that bounded device waits set when they run out. Call it
+ * after synchronizing the stream(s) that ran the kernels. *status_out = MACAQ_OK or
+ * MACAQ_ERR_TIMEOUT. reset != 0 clears the word afterwards. Uses the current CUDA device.
+ * The wait limit can be lowered for tests with macaq_set_wait_limit_ns().
+ */
+macaq_status macaq_device_status(int32_t *status_out, int32_t reset);
+
+/* Sets the time limit of every bounded device-side wait launched after this call (nanoseconds;
+ * 0 restores the default of 2 s). Process-wide. */
+void macaq_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MACAQ_H */

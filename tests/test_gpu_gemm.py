@@ -1,0 +1,211 @@
+"""GPU parity of the W4A4 block-scaled GEMM (dense and grouped).
+
+The fp32 output must match the oracle's float64 sum to within 1e-5 of sum|terms| per element
+(the accumulation order is free); the bf16 output must equal the round-to-nearest-even cast of
+the fp32 output bit for bit. Inputs are either seeded random codes and scales (all 16 codes and a
+spread of scales, independent of the quantizer) or the full pipeline from bf16 X and W, in which
+case each side quantizes with its own code."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w4a4_mxfp4_quantized_b200 as mq
+from w4a4_mxfp4_quantized_b200 import inputs
+from sfutil import Guarded, grouped_sf_rows, sf_index, swizzle
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+
+
+def random_operands(seed, M, N, K, E=None):
+    rng = np.random.default_rng(seed)
+    Aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    Asf = rng.integers(112, 140, (M, K // 32), dtype=np.uint8)
+    shape_w = (N, K // 2) if E is None else (E, N, K // 2)
+    Wq = rng.integers(0, 256, shape_w, dtype=np.uint8)
+    Wsf = rng.integers(112, 140, shape_w[:-1] + (K // 32,), dtype=np.uint8)
+    return Aq, Asf, Wq, Wsf
+
+
+def run_linear(Aq, Asf_tiled, Wq, Wsf_tiled, M, N, out_dtype):
+    Y = Guarded(M * N * (4 if out_dtype == mq.OUT_F32 else 2),
+                dtype=torch.float32 if out_dtype == mq.OUT_F32 else torch.bfloat16, shape=(M, N))
+    mq.linear(Aq, Asf_tiled, Wq, Wsf_tiled, out_dtype=out_dtype, Y=Y.t)
+    torch.cuda.synchronize()
+    assert Y.intact(), "write outside Y"
+    assert mq.device_status() == 0
+    return Y.t
+
+
+def assert_close(y_gpu, Y, T, rows=None):
+    y = y_gpu.double().cpu().numpy()
+    if rows is not None:
+        y = y[rows]
+    err = np.abs(y - Y)
+    bound = RTOL * T + 1e-30
+    bad = np.argwhere(err > bound)
+    assert bad.size == 0, f"{len(bad)} outputs off, worst rel {np.max(err / (T + 1e-30)):.3g} at {bad[:3].tolist()}"
+
+
+def check_dense(Aq, Asf, Wq, Wsf, rows=None):
+    M, N, K = Aq.shape[0], Wq.shape[0], Aq.shape[1] * 2
+    dA = torch.from_numpy(Aq).cuda()
+    dW = torch.from_numpy(Wq).cuda()
+    dAsf = torch.from_numpy(swizzle(Asf, K)).cuda()
+    dWsf = torch.from_numpy(swizzle(Wsf, K)).cuda()
+    y32 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_F32)
+    y16 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_BF16)
+    Y, T = oracle.linear(Aq, Asf, Wq, Wsf, rows=rows)
+    assert_close(y32, Y, T, rows)
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (16, 256, 256), (1, 128, 128), (3, 384, 384), (17, 256, 768), (128, 256, 512),
+    (129, 512, 512), (300, 128, 1024), (256, 768, 4096), (64, 1024, 5120),
+])
+def test_random_codes(M, N, K):
+    check_dense(*random_operands(M * 7 + N + K, M, N, K))
+
+
+def test_extreme_scales_and_codes():
+    """Every code against every code, and scales near both ends of the fp32 product range."""
+    M, N, K = 16, 256, 256
+    Aq = np.tile(np.arange(256, dtype=np.uint8), (M, K // 2 // 256 + 1))[:, :K // 2].copy()
+    Wq = np.roll(np.tile(np.arange(256, dtype=np.uint8), (N, 1))[:, :K // 2], 3, axis=1).copy()
+    Asf = np.full((M, K // 32), 127, np.uint8)
+    Wsf = np.full((N, K // 32), 127, np.uint8)
+    Asf[1] = 160          # 2^33: products up to 2^96 * 36 stay finite in fp32
+    Wsf[:, 1] = 60        # 2^-67
+    Asf[2, 3] = 0         # the smallest scale, 2^-127
+    Wsf[5] = 190          # 2^63
+    Asf[5] = 10           # 2^-117
+    check_dense(Aq, Asf, Wq, Wsf)
+
+
+def pipeline(c, b=32):
+    """Each side quantizes with its own code; returns GPU operands and oracle operands."""
+    s = c.s
+    oWq, oWsf, oinv = oracle.prep_weights(c.W, s, b)
+    oXq, oXsf = oracle.act_quant(c.X, oinv, b)
+    gWq, gWsf, ginv = mq.prep_weights(c.W.cuda(), s.cuda(), b)
+    gXq, gXsf = mq.act_quant(c.X.cuda(), ginv, b)
+    return (gXq, gXsf, gWq, gWsf), (oXq, oXsf, oWq, oWsf)
+
+
+def test_tiny_workload_pipeline():
+    c = inputs.tiny()
+    (gXq, gXsf, gWq, gWsf), (oXq, oXsf, oWq, oWsf) = pipeline(c)
+    M, N = c.X.shape[0], c.W.shape[0]
+    y32 = run_linear(gXq, gXsf, gWq, gWsf, M, N, mq.OUT_F32)
+    y16 = run_linear(gXq, gXsf, gWq, gWsf, M, N, mq.OUT_BF16)
+    Y, T = oracle.linear(oXq, oXsf, oWq, oWsf)
+    assert_close(y32, Y, T)
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+    ref = c.X.double() @ c.W.double().T
+    rel = (y32.double().cpu() - ref).norm() / ref.norm()
+    assert rel < 0.6
+
+
+@pytest.mark.parametrize("M", inputs.LLAMA3_8B_M)
+def test_llama3_8b_up_sampled(M):
+    c = inputs.llama3_8b_up(M)
+    (gXq, gXsf, gWq, gWsf), (oXq, oXsf, oWq, oWsf) = pipeline(c)
+    N = c.W.shape[0]
+    y32 = run_linear(gXq, gXsf, gWq, gWsf, M, N, mq.OUT_F32)
+    y16 = run_linear(gXq, gXsf, gWq, gWsf, M, N, mq.OUT_BF16)
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+    rng = np.random.default_rng(M)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 6)])) if M > 1 else np.array([0])
+    Y, T = oracle.linear(oXq, oXsf, oWq, oWsf, rows=rows)
+    assert_close(y32, Y, T, rows)
+
+
+# ------------------------------------------------------------------------------------- grouped
+def run_grouped(Aq, Asf_t, offsets, Wq, Wsf_t, out_dtype):
+    M = Aq.shape[0]
+    E, N, _ = Wq.shape
+    dt = torch.float32 if out_dtype == mq.OUT_F32 else torch.bfloat16
+    Y = Guarded(M * N * (4 if out_dtype == mq.OUT_F32 else 2), dtype=dt, shape=(M, N))
+    Y.t.zero_()
+    off_d = torch.tensor(np.asarray(offsets, np.int32), device="cuda")
+    mq.grouped_linear(Aq, Asf_t, off_d, Wq, Wsf_t, out_dtype=out_dtype, Y=Y.t)
+    torch.cuda.synchronize()
+    assert Y.intact()
+    assert mq.device_status() == 0
+    return Y.t
+
+
+def grouped_tiled_sf(Asf, offsets, K):
+    rows = grouped_sf_rows(offsets)
+    E = len(offsets) - 1
+    buf = np.zeros(mq.grouped_sf_bytes(Asf.shape[0], E, K), np.uint8)
+    buf[sf_index(rows, K)] = Asf
+    return buf
+
+
+@pytest.mark.parametrize("offsets,N,K", [
+    ([0, 5, 5, 140, 141, 141, 300], 256, 256),
+    ([0, 0, 1, 129, 257, 257], 128, 384),
+    ([0, 64, 64, 64, 200], 512, 1024),
+])
+def test_grouped_random_codes(offsets, N, K):
+    E = len(offsets) - 1
+    M = offsets[-1]
+    Aq, Asf, Wq, Wsf = random_operands(E * 11 + K, M, N, K, E=E)
+    dWsf = torch.from_numpy(np.stack([swizzle(Wsf[e], K) for e in range(E)])).cuda()
+    dAsf = torch.from_numpy(grouped_tiled_sf(Asf, offsets, K)).cuda()
+    dA, dW = torch.from_numpy(Aq).cuda(), torch.from_numpy(Wq).cuda()
+    y32 = run_grouped(dA, dAsf, offsets, dW, dWsf, mq.OUT_F32)
+    y16 = run_grouped(dA, dAsf, offsets, dW, dWsf, mq.OUT_BF16)
+    Y, T = oracle.grouped_linear(Aq, Asf, offsets, Wq, Wsf)
+    assert_close(y32, Y, T)
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+
+
+@pytest.mark.parametrize("T", [64])
+def test_moe_pipeline_sampled(T):
+    c = inputs.moe_30b_a3b(T, "gate_up")
+    E, N, K = c.W.shape
+    off = c.offsets.numpy()
+    oinv = [None] * E
+    oWq = np.empty((E, N, K // 2), np.uint8)
+    oWsf = np.empty((E, N, K // 32), np.uint8)
+    gWq = torch.empty(E, N, K // 2, dtype=torch.uint8, device="cuda")
+    gWsf = torch.empty(E, mq.sf_bytes(N, K), dtype=torch.uint8, device="cuda")
+    ginv = torch.empty(E, K, dtype=torch.float32, device="cuda")
+    Wd = c.W.cuda()
+    sd = c.s.cuda()
+    for e in range(E):
+        oWq[e], oWsf[e], oinv[e] = oracle.prep_weights(c.W[e], c.s[e], 32)
+        mq.prep_weights(Wd[e], sd[e], 32, Wq=gWq[e], Wsf=gWsf[e], inv_s=ginv[e])
+    oinv = np.stack(oinv)
+    oXq, oXsf = oracle.act_quant(c.X, oinv, 32, offsets=off)
+    off_d = c.offsets.cuda()
+    gXq, gXsf = mq.act_quant(c.X.cuda(), ginv, 32, group_offsets=off_d)
+    y32 = run_grouped(gXq, gXsf, off, gWq, gWsf, mq.OUT_F32)
+    rng = np.random.default_rng(T)
+    rows = np.unique(np.concatenate([[0, off[-1] - 1], rng.integers(0, off[-1], 24)]))
+    Y, Tt = oracle.grouped_linear(oXq, oXsf, off, oWq, oWsf, rows=rows)
+    assert_close(y32, Y, Tt, rows)
+
+
+# ------------------------------------------------------------------------------------- failure
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait limit of 1 ns makes the GEMM's first pipeline wait run out: the kernel must return,
+    report MACAQ_ERR_TIMEOUT through the status word, and leave the context usable."""
+    M, N, K = 256, 512, 2048
+    Aq, Asf, Wq, Wsf = random_operands(3, M, N, K)
+    dA, dW = torch.from_numpy(Aq).cuda(), torch.from_numpy(Wq).cuda()
+    dAsf, dWsf = torch.from_numpy(swizzle(Asf, K)).cuda(), torch.from_numpy(swizzle(Wsf, K)).cuda()
+    mq.device_status(reset=True)
+    try:
+        mq.set_wait_limit_ns(1)
+        mq.linear(dA, dAsf, dW, dWsf, out_dtype=mq.OUT_F32)
+        torch.cuda.synchronize()
+    finally:
+        mq.set_wait_limit_ns(0)
+    assert mq.device_status(reset=True) == 6
+    assert mq.device_status() == 0
+    check_dense(Aq, Asf, Wq, Wsf, rows=np.array([0, 100, 255]))

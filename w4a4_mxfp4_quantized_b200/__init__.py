@@ -1,0 +1,216 @@
+"""W4A4 / MXFP4 linear layer of MACaQ on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libmacaq.so`` (C ABI in ``include/macaq.h``). Every function here only
+marshals torch CUDA tensors into pointers and sizes, allocates outputs with torch when the caller
+does not pass them, and raises on a non-zero status: all arithmetic runs in the library's CUDA
+kernels. There is no CPU fallback; calling without the built library raises.
+
+Method (page "Huawei's research lab in Switzerland open-sources the four-bit quantization tool
+MACaQ for running models locally", aipolix.com, paragraphs 2-3; page "MACaQ quantizer from
+huawei-csl targets GGUF, vLLM and Diffusers models", glonce.com, paragraph 5):
+    W' = MXFP4(W diag(s) H_b / b)      prep_weights (offline)
+    X' = MXFP4(X diag(1/s) H_b)        act_quant (online)
+    Y  = X' W'^T                       linear / grouped_linear
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "MacaqError", "OUT_BF16", "OUT_F32", "A_QUANTIZED", "A_BF16_FUSED",
+    "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "status_str",
+    "prep_weights", "act_quant", "linear", "grouped_linear", "device_status", "set_wait_limit_ns",
+    "library_path", "lib",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libmacaq.so")
+_lock = threading.Lock()
+_lib = None
+
+OUT_BF16, OUT_F32 = 0, 1
+A_QUANTIZED, A_BF16_FUSED = 0, 1
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_sz = ctypes.c_size_t
+
+_SIGNATURES = {
+    "macaq_status_str": ([ctypes.c_int], ctypes.c_char_p),
+    "macaq_last_cuda_error": ([], ctypes.c_int),
+    "macaq_sf_bytes": ([_i64, _i64], _sz),
+    "macaq_grouped_sf_bytes": ([_i64, _i32, _i64], _sz),
+    "macaq_workspace_bytes": ([_i64, _i64, _i64, _i32], _sz),
+    "macaq_prep_weights": ([_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "macaq_act_quant": ([_vp, _vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
+    "macaq_linear": ([_i32, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp, _sz, _vp],
+                     ctypes.c_int),
+    "macaq_grouped_linear": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp,
+                              _sz, _vp], ctypes.c_int),
+    "macaq_device_status": ([ctypes.POINTER(ctypes.c_int32), _i32], ctypes.c_int),
+    "macaq_set_wait_limit_ns": ([ctypes.c_uint64], None),
+}
+
+
+class MacaqError(RuntimeError):
+    """A libmacaq call returned a non-zero status."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = status_str(status)
+        extra = ""
+        if name == "MACAQ_ERR_CUDA":
+            extra = f" (cudaError {lib().macaq_last_cuda_error()})"
+        super().__init__(f"{fn} failed: {name}{extra}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded libmacaq.so (raises if it has not been built: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(_LIB_PATH):
+                    raise RuntimeError(
+                        f"libmacaq.so is missing at {_LIB_PATH}; build it with "
+                        "`python -m w4a4_mxfp4_quantized_b200.build` (nvcc, sm_100a)")
+                L = ctypes.CDLL(_LIB_PATH)
+                for name, (args, res) in _SIGNATURES.items():
+                    f = getattr(L, name)
+                    f.argtypes = args
+                    f.restype = res
+                _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().macaq_status_str(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise MacaqError(fn, status)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmacaq takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libmacaq takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def sf_bytes(rows: int, K: int) -> int:
+    """Bytes of the tiled scale-factor buffer of `rows` rows of K elements."""
+    return int(lib().macaq_sf_bytes(rows, K))
+
+
+def grouped_sf_bytes(total_rows: int, E: int, K: int) -> int:
+    return int(lib().macaq_grouped_sf_bytes(total_rows, E, K))
+
+
+def workspace_bytes(M: int, N: int, K: int, E: int = 0) -> int:
+    return int(lib().macaq_workspace_bytes(M, N, K, E))
+
+
+def prep_weights(W: torch.Tensor, s: torch.Tensor | None, had_block: int = 32, *, Wq=None, Wsf=None,
+                 inv_s=None):
+    """Offline W' = MXFP4(W diag(s) H_b / b). Returns (Wq u8 [N, K/2], Wsf u8 tiled, inv_s fp32 [K] or None)."""
+    assert W.dtype == torch.bfloat16 and W.dim() == 2
+    N, K = W.shape
+    dev = W.device
+    Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev) if Wq is None else Wq
+    Wsf = torch.empty(max(sf_bytes(N, K), 16), dtype=torch.uint8, device=dev) if Wsf is None else Wsf
+    if s is not None and inv_s is None:
+        inv_s = torch.empty(K, dtype=torch.float32, device=dev)
+    _check("macaq_prep_weights", lib().macaq_prep_weights(
+        _ptr(W), _ptr(s), N, K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(inv_s) if s is not None else None,
+        _stream(dev)))
+    return Wq, Wsf, (inv_s if s is not None else None)
+
+
+def act_quant(X: torch.Tensor, inv_s: torch.Tensor | None, had_block: int = 32, *, group_offsets=None,
+              Xq=None, Xsf=None):
+    """Online X' = MXFP4(X diag(inv_s) H_b). Returns (Xq u8 [M, K/2], Xsf u8 tiled).
+
+    group_offsets (int32 CUDA [E+1]) selects the grouped form: inv_s is then [E, K]."""
+    assert X.dtype == torch.bfloat16 and X.dim() == 2
+    M, K = X.shape
+    dev = X.device
+    E = 0 if group_offsets is None else group_offsets.numel() - 1
+    Xq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev) if Xq is None else Xq
+    if Xsf is None:
+        n = grouped_sf_bytes(M, E, K) if group_offsets is not None else sf_bytes(M, K)
+        Xsf = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    _check("macaq_act_quant", lib().macaq_act_quant(
+        _ptr(X), _ptr(inv_s), M, K, had_block, _ptr(group_offsets), E, _ptr(Xq), _ptr(Xsf), _stream(dev)))
+    return Xq, Xsf
+
+
+def _out(M, N, out_dtype, dev, Y):
+    if Y is not None:
+        return Y
+    return torch.empty(M, N, dtype=torch.float32 if out_dtype == OUT_F32 else torch.bfloat16, device=dev)
+
+
+def linear(A: torch.Tensor, Asf: torch.Tensor | None, Wq: torch.Tensor, Wsf: torch.Tensor, *,
+           mode: int = A_QUANTIZED, inv_s: torch.Tensor | None = None, had_block: int = 32,
+           out_dtype: int = OUT_BF16, Y=None, workspace=None):
+    """Dense W4A4 linear Y = dq(A) dq(W')^T (fp32 accumulate; bf16 or fp32 out)."""
+    N = Wq.shape[0]
+    K = Wq.shape[1] * 2
+    M = A.shape[0]
+    dev = A.device
+    Y = _out(M, N, out_dtype, dev, Y)
+    ws_need = workspace_bytes(M, N, K, 0)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("macaq_linear", lib().macaq_linear(
+        mode, _ptr(A), _ptr(Asf), _ptr(inv_s), M, N, K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype,
+        _ptr(workspace), ws_bytes, _stream(dev)))
+    return Y
+
+
+def grouped_linear(A: torch.Tensor, Asf: torch.Tensor, group_offsets: torch.Tensor, Wq: torch.Tensor,
+                   Wsf: torch.Tensor, *, out_dtype: int = OUT_BF16, Y=None, workspace=None):
+    """Grouped W4A4 linear: rows of expert e times W'_e. Wq [E, N, K/2], Wsf [E, sf_bytes(N, K)]."""
+    E, N, K2 = Wq.shape
+    K = K2 * 2
+    M = A.shape[0]
+    dev = A.device
+    Y = _out(M, N, out_dtype, dev, Y)
+    ws_need = workspace_bytes(M, N, K, E)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("macaq_grouped_linear", lib().macaq_grouped_linear(
+        A_QUANTIZED, _ptr(A), _ptr(Asf), None, _ptr(group_offsets), E, M, N, K, 32, _ptr(Wq), _ptr(Wsf), _ptr(Y),
+        out_dtype, _ptr(workspace), ws_bytes, _stream(dev)))
+    return Y
+
+
+def device_status(reset: bool = False) -> int:
+    """The sticky device status word (0, or 6 = a bounded wait ran out). Synchronize first."""
+    v = ctypes.c_int32(0)
+    _check("macaq_device_status", lib().macaq_device_status(ctypes.byref(v), 1 if reset else 0))
+    return int(v.value)
+
+
+def set_wait_limit_ns(ns: int):
+    lib().macaq_set_wait_limit_ns(int(ns))

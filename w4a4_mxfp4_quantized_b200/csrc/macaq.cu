@@ -1,0 +1,336 @@
+// macaq.cu -- the C ABI of libmacaq.so (declared in include/macaq.h): argument validation,
+// tensor-map descriptors (cached), and the launches of the quantization and GEMM kernels.
+//
+// Everything is one translation unit so that the device status word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "macaq.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace macaq {
+
+namespace {
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitNs};
+thread_local int t_last_cuda_error = 0;
+
+macaq_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return MACAQ_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_block(int32_t b) { return b == 1 || b == 16 || b == 32 || b == 64 || b == 128; }
+
+// ------------------------------------------------------------------------ device properties
+struct DeviceInfo {
+    int sms = 0;
+    int major = 0;
+    int minor = 0;
+};
+
+macaq_status device_info(DeviceInfo *out) {
+    static std::mutex mu;
+    static std::map<int, DeviceInfo> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(dev);
+    if (it == cache.end()) {
+        DeviceInfo d;
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        it = cache.emplace(dev, d).first;
+    }
+    *out = it->second;
+    if (out->major != 10) return MACAQ_ERR_UNSUPPORTED;  // built for sm_100a only
+    return MACAQ_OK;
+}
+
+// ------------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+using MapKey = std::tuple<int, uintptr_t, int, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t, int>;
+
+// A 2-D tiled tensor map over a row-major matrix: `inner` contiguous elements per row, `outer`
+// rows `row_bytes` apart; box of box_inner x box_outer elements; zero fill out of bounds.
+macaq_status tensor_map_2d(CUtensorMap *out, const void *base, CUtensorMapDataType dtype, uint64_t inner,
+                           uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                           CUtensorMapSwizzle swizzle) {
+    static std::mutex mu;
+    static std::map<MapKey, CUtensorMap> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int>(dtype), inner, outer, row_bytes,
+                     box_inner, box_outer, static_cast<int>(swizzle)};
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *out = it->second;
+        return MACAQ_OK;
+    }
+    auto fn = encode_fn();
+    if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+    CUtensorMap m;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&m, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    if (cache.size() > 4096) cache.clear();
+    cache.emplace(key, m);
+    *out = m;
+    return MACAQ_OK;
+}
+
+template <typename Kernel>
+macaq_status set_smem(Kernel k, size_t bytes) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------------------ quantization
+template <int kB, bool kWeight>
+macaq_status run_quant_b(const CUtensorMap &map, const QuantArgs &a, int grid, cudaStream_t st) {
+    auto k = quant_kernel<kB, kWeight>;
+    const size_t smem = quant_smem_bytes(a.E);
+    macaq_status s = set_smem(k, smem);
+    if (s != MACAQ_OK) return s;
+    k<<<grid, kQThreads, smem, st>>>(map, a);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+}
+
+template <bool kWeight>
+macaq_status run_quant(int32_t b, const CUtensorMap &map, const QuantArgs &a, int grid, cudaStream_t st) {
+    switch (b) {
+        case 1: return run_quant_b<1, kWeight>(map, a, grid, st);
+        case 16: return run_quant_b<16, kWeight>(map, a, grid, st);
+        case 32: return run_quant_b<32, kWeight>(map, a, grid, st);
+        case 64: return run_quant_b<64, kWeight>(map, a, grid, st);
+        case 128: return run_quant_b<128, kWeight>(map, a, grid, st);
+        default: return MACAQ_ERR_UNSUPPORTED;
+    }
+}
+
+macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, int32_t b, bool weight,
+                      const int32_t *offsets, int32_t E, uint8_t *q, uint8_t *sf, float *inv_s, cudaStream_t st) {
+    if (rows < 0 || K <= 0 || K % 128 != 0) return MACAQ_ERR_SHAPE;
+    if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
+    if (offsets != nullptr && (E < 1 || E > 16384)) return MACAQ_ERR_SHAPE;
+    if (rows * (K / 32) >= (int64_t(1) << 31)) return MACAQ_ERR_SHAPE;
+    if (rows == 0 && (inv_s == nullptr || mul == nullptr)) return MACAQ_OK;
+    if (rows > 0 && (X == nullptr || q == nullptr || sf == nullptr)) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(q) || !aligned16(sf) || !aligned16(mul) || !aligned16(inv_s) ||
+        !aligned16(offsets))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+
+    QuantArgs a;
+    a.mul = mul;
+    a.offsets = offsets;
+    a.q = q;
+    a.sf = sf;
+    a.inv_s = inv_s;
+    a.rows = rows;
+    a.K = static_cast<uint32_t>(K);
+    a.kg = static_cast<uint32_t>(K / 32);
+    a.total_groups = static_cast<uint32_t>(rows * (K / 32));
+    a.num_tiles = (a.total_groups + kQGroupsPerTile - 1) / kQGroupsPerTile;
+    a.E = offsets ? E : 1;
+    a.wait_limit_ns = g_wait_limit_ns.load();
+
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof map);
+    if (rows > 0) {
+        // the bf16 matrix as a flat run of 128-byte lines (64 elements), 128 lines per tile
+        const uint64_t lines = static_cast<uint64_t>(rows) * K / 64;
+        s = tensor_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, lines, 128, 64, kQTileLines,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+        if (s != MACAQ_OK) return s;
+    }
+    int grid = static_cast<int>(a.num_tiles);
+    const int max_grid = dev.sms * 3;
+    if (grid > max_grid) grid = max_grid;
+    if (grid < 1) grid = 1;
+    return weight ? run_quant<true>(b, map, a, grid, st) : run_quant<false>(b, map, a, grid, st);
+}
+
+// ------------------------------------------------------------------------ GEMM
+template <int BN, bool kGrouped>
+macaq_status run_gemm(const CUtensorMap &amap, const CUtensorMap &bmap, const GemmArgs &g, dim3 grid,
+                      cudaStream_t st) {
+    auto k = gemm_mxf4_kernel<BN, kGrouped>;
+    const size_t smem = gemm_smem_bytes<BN>(kGrouped ? g.E : 0);
+    macaq_status s = set_smem(k, smem);
+    if (s != MACAQ_OK) return s;
+    k<<<grid, kGemmThreads, smem, st>>>(amap, bmap, g);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+}
+
+macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, int32_t E, int64_t rows, int64_t N,
+                  int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, cudaStream_t st) {
+    if (rows < 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 128 != 0) return MACAQ_ERR_SHAPE;
+    if (rows >= (int64_t(1) << 31) || static_cast<int64_t>(E) * N >= (int64_t(1) << 31)) return MACAQ_ERR_SHAPE;
+    if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
+    if (offsets != nullptr && (E < 1 || E > 1024)) return MACAQ_ERR_SHAPE;
+    if (rows == 0) return MACAQ_OK;
+    if (A == nullptr || Asf == nullptr || Wq == nullptr || Wsf == nullptr || Y == nullptr)
+        return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(Asf) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(Y) ||
+        !aligned16(offsets))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+
+    const int BN = (N % 256 == 0) ? 256 : 128;
+    const bool grouped = offsets != nullptr;
+    const int32_t experts = grouped ? E : 1;
+    GemmArgs g;
+    g.asf = Asf;
+    g.bsf = Wsf;
+    g.y = Y;
+    g.offsets = offsets;
+    g.rows = rows;
+    g.N = static_cast<int32_t>(N);
+    g.K = static_cast<int32_t>(K);
+    g.E = experts;
+    g.out_f32 = out_dtype == MACAQ_OUT_F32;
+    g.bsf_stride = macaq_sf_bytes(N, K);
+    g.wait_limit_ns = g_wait_limit_ns.load();
+
+    CUtensorMap amap, bmap;
+    s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, kBM,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MACAQ_OK) return s;
+    s = tensor_map_2d(&bmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, static_cast<uint64_t>(experts) * N, K / 2,
+                      kBKBytes, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MACAQ_OK) return s;
+
+    const int64_t m_tiles = grouped ? (rows + 127) / 128 + experts : (rows + 127) / 128;
+    if (m_tiles > 65535) return MACAQ_ERR_SHAPE;
+    dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(m_tiles));
+    if (BN == 256) return grouped ? run_gemm<256, true>(amap, bmap, g, grid, st) : run_gemm<256, false>(amap, bmap, g, grid, st);
+    return grouped ? run_gemm<128, true>(amap, bmap, g, grid, st) : run_gemm<128, false>(amap, bmap, g, grid, st);
+}
+
+}  // namespace
+}  // namespace macaq
+
+// ============================================================================ C ABI
+extern "C" {
+
+const char *macaq_status_str(int status) {
+    switch (status) {
+        case MACAQ_OK: return "MACAQ_OK";
+        case MACAQ_ERR_INVALID_ARG: return "MACAQ_ERR_INVALID_ARG";
+        case MACAQ_ERR_SHAPE: return "MACAQ_ERR_SHAPE";
+        case MACAQ_ERR_ALIGNMENT: return "MACAQ_ERR_ALIGNMENT";
+        case MACAQ_ERR_UNSUPPORTED: return "MACAQ_ERR_UNSUPPORTED";
+        case MACAQ_ERR_CUDA: return "MACAQ_ERR_CUDA";
+        case MACAQ_ERR_TIMEOUT: return "MACAQ_ERR_TIMEOUT";
+        case MACAQ_ERR_WORKSPACE: return "MACAQ_ERR_WORKSPACE";
+        default: return "MACAQ_ERR_UNKNOWN";
+    }
+}
+
+int macaq_last_cuda_error(void) { return macaq::t_last_cuda_error; }
+
+size_t macaq_sf_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0 || K % 128 != 0) return 0;
+    return static_cast<size_t>((rows + 127) / 128) * 128 * static_cast<size_t>(K / 32);
+}
+
+size_t macaq_grouped_sf_bytes(int64_t total_rows, int32_t E, int64_t K) {
+    if (total_rows < 0 || E < 0 || K <= 0 || K % 128 != 0) return 0;
+    return static_cast<size_t>((total_rows + 127) / 128 + E) * 128 * static_cast<size_t>(K / 32);
+}
+
+size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E) {
+    (void)M, (void)N, (void)K, (void)E;
+    return 0;
+}
+
+macaq_status macaq_prep_weights(const void *W, const float *s, int64_t N, int64_t K, int32_t had_block, uint8_t *Wq,
+                                uint8_t *Wsf, float *inv_s, macaq_stream_t stream) {
+    if (N % 128 != 0) return MACAQ_ERR_SHAPE;
+    return macaq::quantize(W, s, N, K, had_block, true, nullptr, 0, Wq, Wsf, s ? inv_s : nullptr,
+                           static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64_t K, int32_t had_block,
+                             const int32_t *group_offsets, int32_t E, uint8_t *Xq, uint8_t *Xsf,
+                             macaq_stream_t stream) {
+    return macaq::quantize(X, inv_s, M, K, had_block, false, group_offsets, E, Xq, Xsf, nullptr,
+                           static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M, int64_t N,
+                          int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
+                          int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
+    (void)inv_s, (void)had_block, (void)workspace, (void)ws_bytes;
+    if (mode == MACAQ_A_BF16_FUSED) return MACAQ_ERR_UNSUPPORTED;
+    if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
+    return macaq::gemm(static_cast<const uint8_t *>(A), Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype,
+                       static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
+                                  const int32_t *group_offsets, int32_t E, int64_t total_rows, int64_t N, int64_t K,
+                                  int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
+                                  int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
+    (void)inv_s, (void)had_block, (void)workspace, (void)ws_bytes;
+    if (mode != MACAQ_A_QUANTIZED) return mode == MACAQ_A_BF16_FUSED ? MACAQ_ERR_UNSUPPORTED : MACAQ_ERR_INVALID_ARG;
+    if (group_offsets == nullptr) return MACAQ_ERR_INVALID_ARG;
+    return macaq::gemm(static_cast<const uint8_t *>(A), Asf, group_offsets, E, total_rows, N, K, Wq, Wsf, Y,
+                       out_dtype, static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_device_status(int32_t *status_out, int32_t reset) {
+    if (status_out == nullptr) return MACAQ_ERR_INVALID_ARG;
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, macaq::g_device_status, sizeof v);
+    if (e != cudaSuccess) return macaq::cuda_fail(e);
+    *status_out = v;
+    if (reset) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(macaq::g_device_status, &zero, sizeof zero);
+        if (e != cudaSuccess) return macaq::cuda_fail(e);
+    }
+    return MACAQ_OK;
+}
+
+void macaq_set_wait_limit_ns(uint64_t ns) { macaq::g_wait_limit_ns.store(ns ? ns : macaq::kDefaultWaitNs); }
+
+}  // extern "C"
