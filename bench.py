@@ -48,6 +48,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--M", type=int, default=M_MAIN)
     p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--profile", action="store_true", help="eager passes only, for ncu captures")
     return p.parse_args()
 
 
@@ -129,16 +130,19 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------ our arm
-def make_layer(M, dev, copies):
+def make_layer(M, dev, copies, plain=False):
+    """The layer's device buffers. plain=True is the plain-MXFP4 comparator: no per-channel scale
+    and no Hadamard (block 1), same kernels and shapes."""
     import w4a4_mxfp4_quantized_b200 as mq
     from w4a4_mxfp4_quantized_b200 import inputs
 
     c = inputs.llama3_8b_up(M)
     W = c.W.to(dev)
-    s = c.s.to(dev)
+    s = None if plain else c.s.to(dev)
+    b = 1 if plain else HAD_BLOCK
     Xs = [c.X.to(dev)]
     Wqs, Wsfs = [], []
-    Wq, Wsf, inv_s = mq.prep_weights(W, s, HAD_BLOCK)
+    Wq, Wsf, inv_s = mq.prep_weights(W, s, b)
     Wqs.append(Wq)
     Wsfs.append(Wsf)
     for _ in range(copies - 1):
@@ -149,7 +153,7 @@ def make_layer(M, dev, copies):
     Xq = [torch.empty(M, K_DIM // 2, dtype=torch.uint8, device=dev) for _ in range(copies)]
     Xsf = [torch.empty(mq.sf_bytes(M, K_DIM), dtype=torch.uint8, device=dev) for _ in range(copies)]
     Y = [torch.empty(M, N_DIM, dtype=torch.bfloat16, device=dev) for _ in range(copies)]
-    return dict(X=Xs, inv_s=inv_s, Wq=Wqs, Wsf=Wsfs, Xq=Xq, Xsf=Xsf, Y=Y, host_X=c.X)
+    return dict(X=Xs, inv_s=inv_s, Wq=Wqs, Wsf=Wsfs, Xq=Xq, Xsf=Xsf, Y=Y, host_X=c.X, b=b)
 
 
 def copies_for(M):
@@ -157,43 +161,70 @@ def copies_for(M):
     return max(2, int(np.ceil(2 * L2_BYTES / per_copy)))
 
 
-def run_layer(mq, L, i):
-    mq.act_quant(L["X"][i], L["inv_s"], HAD_BLOCK, Xq=L["Xq"][i], Xsf=L["Xsf"][i])
-    mq.linear(L["Xq"][i], L["Xsf"][i], L["Wq"][i], L["Wsf"][i], Y=L["Y"][i])
+def run_layer(mq, L, i, parts=("aq", "gemm")):
+    if "aq" in parts:
+        mq.act_quant(L["X"][i], L["inv_s"], L["b"], Xq=L["Xq"][i], Xsf=L["Xsf"][i])
+    if "gemm" in parts:
+        mq.linear(L["Xq"][i], L["Xsf"][i], L["Wq"][i], L["Wsf"][i], Y=L["Y"][i])
 
 
-def time_layer(M, steps, warmup, dev, dist_on):
-    """Device time of `steps` layer passes (rotating copies), and per-kernel event times."""
+def capture(mq, L, steps, ncopy, parts):
+    """One CUDA graph holding `steps` passes (rotating over the input copies): replaying it times
+    the kernels alone, without the per-call host overhead of the Python binding."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            run_layer(mq, L, i % ncopy, parts)
+    return g
+
+
+def replay_ms(g, stream):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def time_layer(M, steps, warmup, dev, dist_on, plain=False):
+    """Device time of `steps` layer passes (graph replay, rotating copies) and of each kernel alone."""
     import w4a4_mxfp4_quantized_b200 as mq
 
     ncopy = copies_for(M)
-    L = make_layer(M, dev, ncopy)
-    stream = torch.cuda.current_stream(dev)
-    for i in range(warmup):
+    L = make_layer(M, dev, ncopy, plain)
+    for i in range(max(warmup, 1)):
         run_layer(mq, L, i % ncopy)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    g_pair = capture(mq, L, steps, ncopy, ("aq", "gemm"))
+    g_aq = capture(mq, L, steps, ncopy, ("aq",))
+    g_gemm = capture(mq, L, steps, ncopy, ("gemm",))
+    stream = torch.cuda.current_stream(dev)
+    for g in (g_pair, g_aq, g_gemm):  # warm replays
+        g.replay()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    start.record(stream)
-    for i in range(steps):
-        j = i % ncopy
-        ev[i][0].record(stream)
-        mq.act_quant(L["X"][j], L["inv_s"], HAD_BLOCK, Xq=L["Xq"][j], Xsf=L["Xsf"][j])
-        ev[i][1].record(stream)
-        mq.linear(L["Xq"][j], L["Xsf"][j], L["Wq"][j], L["Wsf"][j], Y=L["Y"][j])
-        ev[i][2].record(stream)
-    stop.record(stream)
-    torch.cuda.synchronize(dev)
+    total_ms = replay_ms(g_pair, stream)
     if dist_on:
         torch.distributed.barrier()
-    total_ms = start.elapsed_time(stop)
-    aq_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    gemm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    aq_ms = replay_ms(g_aq, stream) / steps
+    gemm_ms = replay_ms(g_gemm, stream) / steps
     status = mq.device_status()
     assert status == 0, f"device status {status}"
+    del g_pair, g_aq, g_gemm
     return total_ms, aq_ms, gemm_ms, L
+
+
+def profile_mode(M, steps, warmup, dev):
+    """Eager layer passes with no timing: the command the ncu captures run."""
+    import w4a4_mxfp4_quantized_b200 as mq
+
+    L = make_layer(M, dev, 2)
+    for i in range(warmup + steps):
+        run_layer(mq, L, i % 2)
+    torch.cuda.synchronize(dev)
+    assert mq.device_status() == 0
 
 
 def time_e2e(M, steps, warmup, dev, L):
@@ -285,6 +316,9 @@ def main():
     torch.cuda.set_device(dev)
 
     M = args.M
+    if args.profile:
+        profile_mode(M, args.steps, args.warmup, dev)
+        return
     flops = 2.0 * M * N_DIM * K_DIM
     with ClockSampler(local) as clk:
         total_ms, aq_ms, gemm_ms, L = time_layer(M, args.steps, args.warmup, dev, dist_on)
@@ -295,6 +329,13 @@ def main():
     ms_step = t.item() / args.steps
     value = world * flops / (ms_step * 1e-3) / 1e12
 
+    del L
+    p_total, p_aq, p_gemm, _ = time_layer(M, args.steps, args.warmup, dev, dist_on, plain=True)
+    overhead = {"plain_mxfp4_ms_per_step": p_total / args.steps, "plain_act_quant_ms": p_aq, "plain_gemm_ms": p_gemm,
+                "B_vs_plain_mxfp4_pipeline": (total_ms / args.steps) / (p_total / args.steps) - 1.0,
+                "A_vs_gemm_on_prequantized_A": (total_ms / args.steps) / p_gemm - 1.0,
+                "pages_figure_for_context": "2.3% end-to-end, Qwen3-32B in vLLM, hardware not stated"}
+    _, _, _, L = time_layer(M, 3, 1, dev, dist_on)
     e2e_ms, h2d, d2h = time_e2e(M, max(3, args.steps // 2), 2, dev, L)
     e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
 
@@ -339,6 +380,7 @@ def main():
                 "ms_per_step": e2e_ms},
         "clocks": clocks,
         "sweep": sweep,
+        "transform_overhead": overhead,
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
     print(json.dumps(out))

@@ -136,3 +136,21 @@ def test_prep_weights_blocks(b):
 def test_prep_weights_llama3_8b_up():
     c = inputs.llama3_8b_up(1)
     _check_prep(c.W, c.s, 32)
+
+
+def test_repeated_runs_stay_bit_exact():
+    """Many tiles per CTA and a congested load queue: stage reuse must never let a TMA refill a
+    shared-memory stage before every lane has read it (five repeats of two such workloads)."""
+    c = inputs.llama3_8b_up(1)
+    oq, osf, _ = oracle.prep_weights(c.W, c.s, 32)
+    Wd, sd = c.W.cuda(), c.s.cuda()
+    m = inputs.moe_30b_a3b(1024, "gate_up", draw_w=False)
+    inv = (np.float32(1.0) / m.s.numpy()).astype(np.float32)
+    mq_ref, _ = oracle.act_quant(m.X, inv, 32, offsets=m.offsets.numpy())
+    Xd, invd, offd = m.X.cuda(), torch.from_numpy(inv).cuda(), m.offsets.cuda()
+    for _ in range(5):
+        gq, _, _ = mq.prep_weights(Wd, sd, 32)
+        xq, _ = mq.act_quant(Xd, invd, 32, group_offsets=offd)
+        torch.cuda.synchronize()
+        assert np.array_equal(gq.cpu().numpy(), oq)
+        assert np.array_equal(xq.cpu().numpy(), mq_ref)

@@ -6,16 +6,22 @@
 // (MoE) forms; the grouped form maps each 128-row tile to its expert from the device-side offsets.
 // Source: glonce.com page on MACaQ, paragraph 5 (W4A4 dense and grouped matmul kernels).
 //
-// One CTA computes a 128 x BN output tile. Warp roles (192 threads):
+// Persistent kernel: one CTA per SM walks output tiles of 128 x BN (BN = 256, or 128 when
+// N % 256 != 0) in a grouped raster (bands of kRasterM row tiles) so that the operands of the tiles
+// in flight stay in L2. Warp roles (192 threads):
 //   warp 0      TMA producer: per K-block of 256 elements, the A tile (128 rows x 128 bytes) and the
 //               B tile (BN rows x 128 bytes) with 128-byte swizzle via tensor maps, plus the matching
-//               scale-factor tiles (already in the tcgen05 128x4 tiling) by plain bulk copies;
-//   warp 1      TMEM allocator and MMA issuer: copies the scale factors into TMEM (tcgen05.cp
-//               32x128b.warpx4), then issues 4 MMAs of 128 x BN x 64, and frees the stage with
-//               tcgen05.commit;
-//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator (each warp reads its 32-lane quarter),
-//               conversion and row stores.
-// Stages form an mbarrier ring; every wait is bounded and a timeout leaves the kernel cleanly.
+//               scale-factor tiles (already in the tcgen05 128x4 tiling) by plain bulk copies. It runs
+//               ahead across tile boundaries, limited only by the stage ring.
+//   warp 1      TMEM allocator and MMA issuer: waits until the epilogue has drained the accumulator,
+//               then per K-block copies the scale factors into TMEM (tcgen05.cp 32x128b.warpx4),
+//               issues 4 MMAs of 128 x BN x 64 and frees the stage with tcgen05.commit; a final commit
+//               per tile signals the epilogue.
+//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator (each warp reads its 32-lane quarter);
+//               for bf16 output the whole row is pulled into registers and the accumulator released
+//               before the global stores, so the next tile's MMAs overlap the stores.
+// Every wait is bounded; a timeout anywhere stops all roles of the CTA, lets its own copies and
+// MMAs land, frees TMEM and returns.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -28,6 +34,7 @@ namespace macaq {
 constexpr int kBM = 128;
 constexpr int kBKBytes = 128;  // 256 FP4 elements per K-block
 constexpr int kGemmThreads = 192;
+constexpr int kRasterM = 16;   // row tiles per raster band
 constexpr uint64_t kDrainLimitNs = 2000000000ull;  // waits for the kernel's own copies / MMAs to land
 
 template <int BN>
@@ -65,6 +72,33 @@ __host__ __device__ constexpr size_t gemm_smem_bytes(int E) {
     return GemmCfg<BN>::kSmemBytes + 2 * sizeof(int32_t) * (E + 1);
 }
 
+// Bounded wait that also gives up as soon as another role of the CTA has failed.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                                   volatile int *abort) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(a, parity)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            record_timeout();
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// Tile index -> (row tile, column tile) in bands of kRasterM row tiles, columns inner.
+__device__ __forceinline__ void raster(uint32_t t, uint32_t m_tiles, uint32_t n_tiles, uint32_t &mt, uint32_t &nt) {
+    const uint32_t band = t / (kRasterM * n_tiles);
+    const uint32_t first = band * kRasterM;
+    const uint32_t height = min(static_cast<uint32_t>(kRasterM), m_tiles - first);
+    const uint32_t r = t - band * kRasterM * n_tiles;
+    mt = first + r % height;
+    nt = r / height;
+}
+
 template <int BN, bool kGrouped>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, GemmArgs g) {
@@ -73,9 +107,10 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     extern __shared__ uint8_t dsmem[];
     __shared__ uint64_t full_bar[S];
     __shared__ uint64_t empty_bar[S];
-    __shared__ uint64_t accum_bar;
+    __shared__ uint64_t accum_full;   // MMA -> epilogue: the tile's accumulator is final
+    __shared__ uint64_t accum_empty;  // epilogue -> MMA: the accumulator has been read out
     __shared__ uint32_t tmem_slot;
-    __shared__ volatile int mma_failed;  // set by the MMA thread when it stops early
+    __shared__ volatile int failed;   // set by any role whose wait ran out
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
@@ -87,37 +122,21 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_tile = blockIdx.x;
-    const int m_tile = blockIdx.y;
 
-    // ---- which rows this CTA owns
-    int64_t row0, row_end;
-    int expert = 0;
-    if constexpr (kGrouped) {
-        load_group_layout(g.offsets, g.E, g.rows, s_off, s_tb);  // block-wide
-        if (m_tile >= s_tb[g.E]) return;                         // beyond the last expert's tiles
-        int lo = 0, hi = g.E;                                    // s_tb[lo] <= m_tile < s_tb[hi]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (s_tb[mid] <= m_tile) lo = mid;
-            else hi = mid;
-        }
-        expert = lo;
-        row0 = s_off[expert] + static_cast<int64_t>(m_tile - s_tb[expert]) * kBM;
-        row_end = s_off[expert + 1];
-    } else {
-        row0 = static_cast<int64_t>(m_tile) * kBM;
-        row_end = g.rows;
-    }
-    if (row_end > row0 + kBM) row_end = row0 + kBM;
+    load_group_layout(kGrouped ? g.offsets : nullptr, kGrouped ? g.E : 1, g.rows, s_off, s_tb);  // block-wide
+    const uint32_t m_tiles = static_cast<uint32_t>(s_tb[kGrouped ? g.E : 1]);
+    const uint32_t n_tiles = static_cast<uint32_t>(g.N / BN);
+    const uint32_t num_tiles = m_tiles * n_tiles;
+    if (blockIdx.x >= num_tiles) return;  // uniform across the CTA
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&accum_bar, 1);
-        mma_failed = 0;
+        mbar_init(&accum_full, 1);
+        mbar_init(&accum_empty, 4);  // one arrival per epilogue warp
+        failed = 0;
         fence_mbar_init();
         prefetch_tensor_map(&amap);
         prefetch_tensor_map(&bmap);
@@ -136,100 +155,171 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     const int num_kb = (K + 255) / 256;
     const uint64_t limit = g.wait_limit_ns;
 
+    // Which rows a row tile covers: its expert, first row, row bound.
+    auto tile_rows = [&](uint32_t mt, int &expert, int64_t &row0, int64_t &row_end) {
+        if constexpr (kGrouped) {
+            int lo = 0, hi = g.E;  // s_tb[lo] <= mt < s_tb[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (static_cast<uint32_t>(s_tb[mid]) <= mt) lo = mid;
+                else hi = mid;
+            }
+            expert = lo;
+            row0 = s_off[lo] + static_cast<int64_t>(mt - s_tb[lo]) * kBM;
+            row_end = s_off[lo + 1];
+        } else {
+            expert = 0;
+            row0 = static_cast<int64_t>(mt) * kBM;
+            row_end = g.rows;
+        }
+        if (row_end > row0 + kBM) row_end = row0 + kBM;
+    };
+
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ TMA producer
-            const uint8_t *asf = g.asf + static_cast<uint64_t>(m_tile) * kq * 512;
-            const uint8_t *bsf = g.bsf + static_cast<uint64_t>(expert) * g.bsf_stride +
-                                 static_cast<uint64_t>(n_tile) * (BN / 128) * kq * 512;
-            const int32_t brow = expert * g.N + n_tile * BN;
-            int kb = 0;
-            for (; kb < num_kb; ++kb) {
-                const int s = kb % S;
-                if (kb >= S && !mbar_wait(&empty_bar[s], ((kb / S) & 1) ^ 1, limit)) break;
-                const int kch = (K - kb * 256) >= 256 ? 2 : 1;   // 128-element scale chunks in this block
-                mbar_arrive_expect_tx(&full_bar[s], C::kABytes + C::kBBytes + kch * 512 * (1 + BN / 128));
-                tma_load_2d(sA + s * C::kABytes, &amap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(row0));
-                tma_load_2d(sB + s * C::kBBytes, &bmap, &full_bar[s], kb * kBKBytes, brow);
-                bulk_load(sSfa + s * C::kSfaBytes, asf + kb * 1024, kch * 512, &full_bar[s]);
+            uint32_t j = 0;  // global K-block counter across tiles (stage = j % S)
+            bool stop = false;
+            for (uint32_t t = blockIdx.x; t < num_tiles && !stop; t += gridDim.x) {
+                uint32_t mt, nt;
+                raster(t, m_tiles, n_tiles, mt, nt);
+                int expert;
+                int64_t row0, row_end;
+                tile_rows(mt, expert, row0, row_end);
+                const uint8_t *asf = g.asf + static_cast<uint64_t>(mt) * kq * 512;
+                const uint8_t *bsf = g.bsf + static_cast<uint64_t>(expert) * g.bsf_stride +
+                                     static_cast<uint64_t>(nt) * (BN / 128) * kq * 512;
+                const int32_t brow = expert * g.N + static_cast<int32_t>(nt) * BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++j) {
+                    const int s = j % S;
+                    if (j >= S && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) {
+                        stop = true;
+                        break;
+                    }
+                    const int kch = (K - kb * 256) >= 256 ? 2 : 1;  // 128-element scale chunks in this block
+                    mbar_arrive_expect_tx(&full_bar[s], C::kABytes + C::kBBytes + kch * 512 * (1 + BN / 128));
+                    tma_load_2d(sA + s * C::kABytes, &amap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(row0));
+                    tma_load_2d(sB + s * C::kBBytes, &bmap, &full_bar[s], kb * kBKBytes, brow);
+                    bulk_load(sSfa + s * C::kSfaBytes, asf + kb * 1024, kch * 512, &full_bar[s]);
 #pragma unroll
-                for (int h = 0; h < BN / 128; ++h)
-                    bulk_load(sSfb + s * C::kSfbBytes + h * 1024, bsf + static_cast<uint64_t>(h) * kq * 512 + kb * 1024,
-                              kch * 512, &full_bar[s]);
+                    for (int h = 0; h < BN / 128; ++h)
+                        bulk_load(sSfb + s * C::kSfbBytes + h * 1024, bsf + static_cast<uint64_t>(h) * kq * 512 + kb * 1024,
+                                  kch * 512, &full_bar[s]);
+                }
             }
             // let the copies this thread issued land before the CTA can exit
-            for (int j = (kb > S ? kb - S : 0); j < kb; ++j)
-                if (!mbar_wait(&full_bar[j % S], (j / S) & 1, kDrainLimitNs)) break;
+            for (uint32_t i = (j > S ? j - S : 0); i < j; ++i)
+                if (!mbar_wait(&full_bar[i % S], (i / S) & 1, kDrainLimitNs)) break;
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
             const uint32_t idesc_lo = idesc_mxf4(BN, 0);  // scale bytes 0-1 of each TMEM column
             const uint32_t idesc_hi = idesc_mxf4(BN, 2);  // scale bytes 2-3
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % S;
-                if (!mbar_wait(&full_bar[s], (kb / S) & 1, limit)) {
-                    mma_failed = 1;
-                    __threadfence_block();
+            uint32_t j = 0;
+            uint32_t tiles_done = 0;
+            bool stop = false;
+            for (uint32_t t = blockIdx.x; t < num_tiles && !stop; t += gridDim.x, ++tiles_done) {
+                // the epilogue must have read the previous tile's accumulator out of TMEM
+                if (tiles_done > 0 && !mbar_wait_or_abort(&accum_empty, (tiles_done - 1) & 1, limit, &failed)) {
+                    stop = true;
                     break;
                 }
                 tc_fence_after();
-                const int kch = (K - kb * 256) >= 256 ? 2 : 1;
-                for (int c = 0; c < kch; ++c) {
-                    tc_cp_sf(tmem + C::kTmemSfa + 4 * c, sdesc_sf(smem_u32(sSfa + s * C::kSfaBytes + c * 512)));
+                for (int kb = 0; kb < num_kb; ++kb, ++j) {
+                    const int s = j % S;
+                    if (!mbar_wait_or_abort(&full_bar[s], (j / S) & 1, limit, &failed)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int kch = (K - kb * 256) >= 256 ? 2 : 1;
+                    for (int c = 0; c < kch; ++c) {
+                        tc_cp_sf(tmem + C::kTmemSfa + 4 * c, sdesc_sf(smem_u32(sSfa + s * C::kSfaBytes + c * 512)));
 #pragma unroll
-                    for (int h = 0; h < BN / 128; ++h)
-                        tc_cp_sf(tmem + C::kTmemSfb + c * (BN / 32) + 4 * h,
-                                 sdesc_sf(smem_u32(sSfb + s * C::kSfbBytes + h * 1024 + c * 512)));
+                        for (int h = 0; h < BN / 128; ++h)
+                            tc_cp_sf(tmem + C::kTmemSfb + c * (BN / 32) + 4 * h,
+                                     sdesc_sf(smem_u32(sSfb + s * C::kSfbBytes + h * 1024 + c * 512)));
+                    }
+                    const uint64_t adesc = sdesc_sw128(smem_u32(sA + s * C::kABytes));
+                    const uint64_t bdesc = sdesc_sw128(smem_u32(sB + s * C::kBBytes));
+                    for (int q = 0; q < 2 * kch; ++q) {
+                        const int c = q >> 1;
+                        // K step q covers bytes [32q, 32q + 32) of every 128-byte row
+                        tc_mma_mxf4(tmem, adesc + 2 * q, bdesc + 2 * q, (q & 1) ? idesc_hi : idesc_lo,
+                                    tmem + C::kTmemSfa + 4 * c, tmem + C::kTmemSfb + c * (BN / 32),
+                                    (kb | q) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty_bar[s]);
                 }
-                const uint64_t adesc = sdesc_sw128(smem_u32(sA + s * C::kABytes));
-                const uint64_t bdesc = sdesc_sw128(smem_u32(sB + s * C::kBBytes));
-                for (int j = 0; j < 2 * kch; ++j) {
-                    const int c = j >> 1;
-                    // K step j covers bytes [32j, 32j + 32) of every 128-byte row
-                    tc_mma_mxf4(tmem, adesc + 2 * j, bdesc + 2 * j, (j & 1) ? idesc_hi : idesc_lo,
-                                tmem + C::kTmemSfa + 4 * c, tmem + C::kTmemSfb + c * (BN / 32),
-                                (kb | j) != 0 ? 1u : 0u);
-                }
-                tc_commit(&empty_bar[s]);
+                tc_commit(&accum_full);  // the accumulator is final once every MMA above completed
             }
-            tc_commit(&accum_bar);  // the accumulator is final once every MMA above completed
-            // TMEM is released at the end: make sure no MMA of this thread is still running then
-            mbar_wait(&accum_bar, 0, kDrainLimitNs);
+            // TMEM is released at the end: make sure no MMA of this thread is still running then.
+            // The last commit is this phase's; if the loop stopped before any commit of the current
+            // tile, commit once more so that the wait below covers everything issued.
+            if (stop) {
+                tc_commit(&accum_full);
+                ++tiles_done;
+            }
+            if (tiles_done > 0) mbar_wait(&accum_full, (tiles_done - 1) & 1, kDrainLimitNs);
         }
     } else {
         // ---------------------------------------------------------------- epilogue
-        const int quarter = warp & 3;                        // TMEM lanes this warp may read
+        const int quarter = warp & 3;  // TMEM lanes this warp may read
         const int r = quarter * 32 + lane;
-        const bool ready = mbar_wait(&accum_bar, 0, limit);
-        tc_fence_after();
-        const int64_t row = row0 + r;
-        const bool live = ready && !mma_failed && row < row_end;
-        const int64_t col0 = static_cast<int64_t>(n_tile) * BN;
-#pragma unroll 1
-        for (int cb = 0; cb < BN / 32; ++cb) {
-            uint32_t v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + cb * 32, v);
-            tmem_ld_wait();
-            if (!live) continue;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        uint32_t tiles_done = 0;
+        for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tiles_done) {
+            uint32_t mt, nt;
+            raster(t, m_tiles, n_tiles, mt, nt);
+            int expert;
+            int64_t row0, row_end;
+            tile_rows(mt, expert, row0, row_end);
+            if (!mbar_wait_or_abort(&accum_full, tiles_done & 1, limit, &failed)) break;
+            tc_fence_after();
+            if (failed) break;
+            const int64_t row = row0 + r;
+            const bool live = row < row_end;
+            const int64_t col0 = static_cast<int64_t>(nt) * BN;
             if (g.out_f32) {
-                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(g.y) + row * g.N + col0 + cb * 32);
+                // fp32 (checking) output: read and store 32 columns at a time, then release TMEM
+#pragma unroll 1
+                for (int cb = 0; cb < BN / 32; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + cb * 32, v);
+                    tmem_ld_wait();
+                    if (!live) continue;
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(g.y) + row * g.N + col0 + cb * 32);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accum_empty);
             } else {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(g.y) + row * g.N + col0 + cb * 32);
+                // bf16 output: pull the whole row into registers, release TMEM, then store
+                uint32_t packed[BN / 2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    uint32_t p[4];
+                for (int cb = 0; cb < BN / 32; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + cb * 32, v);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2 * k]),
-                                                                  __uint_as_float(v[8 * i + 2 * k + 1]));
-                        p[k] = *reinterpret_cast<uint32_t *>(&b2);
+                    for (int k = 0; k < 16; ++k) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                        packed[cb * 16 + k] = *reinterpret_cast<uint32_t *>(&b2);
                     }
-                    dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accum_empty);
+                if (live) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(g.y) + row * g.N + col0);
+#pragma unroll
+                    for (int i = 0; i < BN / 8; ++i)
+                        dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
                 }
             }
         }

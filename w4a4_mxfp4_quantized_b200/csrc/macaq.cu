@@ -75,19 +75,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-using MapKey = std::tuple<int, uintptr_t, int, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t, int>;
+using MapKey = std::tuple<int, uintptr_t, int, int, uint64_t, uint64_t, uint64_t, uint64_t, uint64_t, uint32_t,
+                          uint32_t, uint32_t, int>;
 
-// A 2-D tiled tensor map over a row-major matrix: `inner` contiguous elements per row, `outer`
-// rows `row_bytes` apart; box of box_inner x box_outer elements; zero fill out of bounds.
-macaq_status tensor_map_2d(CUtensorMap *out, const void *base, CUtensorMapDataType dtype, uint64_t inner,
-                           uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                           CUtensorMapSwizzle swizzle) {
+// A tiled tensor map of rank 2 or 3 over a strided array: dims[0] contiguous elements, dims[1] and
+// dims[2] with byte strides strides[0] and strides[1]; box of box[0] x box[1] (x box[2]) elements;
+// zero fill out of bounds. Descriptors are cached by everything they encode.
+macaq_status tensor_map(CUtensorMap *out, const void *base, CUtensorMapDataType dtype, int rank,
+                        const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                        CUtensorMapSwizzle swizzle) {
     static std::mutex mu;
     static std::map<MapKey, CUtensorMap> cache;
     int dev = 0;
     cudaGetDevice(&dev);
-    const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int>(dtype), inner, outer, row_bytes,
-                     box_inner, box_outer, static_cast<int>(swizzle)};
+    const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int>(dtype), rank, dims[0], dims[1],
+                     rank > 2 ? dims[2] : 0, strides[0], rank > 2 ? strides[1] : 0, box[0], box[1],
+                     rank > 2 ? box[2] : 0, static_cast<int>(swizzle)};
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end()) {
@@ -97,12 +100,13 @@ macaq_status tensor_map_2d(CUtensorMap *out, const void *base, CUtensorMapDataTy
     auto fn = encode_fn();
     if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
     CUtensorMap m;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(&m, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    cuuint64_t d[3] = {dims[0], dims[1], rank > 2 ? dims[2] : 1};
+    cuuint64_t s[2] = {strides[0], rank > 2 ? strides[1] : 0};
+    cuuint32_t b[3] = {box[0], box[1], rank > 2 ? box[2] : 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&m, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d, s, b, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     if (cache.size() > 4096) cache.clear();
     cache.emplace(key, m);
@@ -110,10 +114,30 @@ macaq_status tensor_map_2d(CUtensorMap *out, const void *base, CUtensorMapDataTy
     return MACAQ_OK;
 }
 
+macaq_status tensor_map_2d(CUtensorMap *out, const void *base, CUtensorMapDataType dtype, uint64_t inner,
+                           uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                           CUtensorMapSwizzle swizzle) {
+    const uint64_t dims[2] = {inner, outer};
+    const uint64_t strides[1] = {row_bytes};
+    const uint32_t box[2] = {box_inner, box_outer};
+    return tensor_map(out, base, dtype, 2, dims, strides, box, swizzle);
+}
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device, size).
 template <typename Kernel>
 macaq_status set_smem(Kernel k, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, int>, size_t> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const auto key = std::make_tuple(reinterpret_cast<const void *>(k), dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find(key);
+    if (it != done.end() && it->second >= bytes) return MACAQ_OK;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+    if (e != cudaSuccess) return cuda_fail(e);
+    done[key] = bytes;
+    return MACAQ_OK;
 }
 
 // ------------------------------------------------------------------------ quantization
@@ -164,24 +188,29 @@ macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, 
     a.rows = rows;
     a.K = static_cast<uint32_t>(K);
     a.kg = static_cast<uint32_t>(K / 32);
-    a.total_groups = static_cast<uint32_t>(rows * (K / 32));
-    a.num_tiles = (a.total_groups + kQGroupsPerTile - 1) / kQGroupsPerTile;
+    a.slab_groups = a.kg % 32 == 0 ? 32 : a.kg % 16 == 0 ? 16 : a.kg % 8 == 0 ? 8 : 4;
+    a.slab_shift = a.slab_groups == 32 ? 5 : a.slab_groups == 16 ? 4 : a.slab_groups == 8 ? 3 : 2;
+    a.slabs = a.kg / a.slab_groups;
+    a.tile_rows = kQConsumers / a.slab_groups;
+    a.row_tiles = static_cast<uint32_t>((rows + a.tile_rows - 1) / a.tile_rows);
     a.E = offsets ? E : 1;
     a.wait_limit_ns = g_wait_limit_ns.load();
 
     CUtensorMap map;
     std::memset(&map, 0, sizeof map);
     if (rows > 0) {
-        // the bf16 matrix as a flat run of 128-byte lines (64 elements), 128 lines per tile
-        const uint64_t lines = static_cast<uint64_t>(rows) * K / 64;
-        s = tensor_map_2d(&map, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, lines, 128, 64, kQTileLines,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+        // X as [rows][K/64 chunks of 128 bytes][64 elements]; a tile is tile_rows x slab x 64
+        const uint64_t dims[3] = {64, static_cast<uint64_t>(K) / 64, static_cast<uint64_t>(rows)};
+        const uint64_t strides[2] = {128, static_cast<uint64_t>(K) * 2};
+        const uint32_t box[3] = {64, a.slab_groups / 2, a.tile_rows};
+        s = tensor_map(&map, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (s != MACAQ_OK) return s;
     }
-    int grid = static_cast<int>(a.num_tiles);
-    const int max_grid = dev.sms * 3;
-    if (grid > max_grid) grid = max_grid;
-    if (grid < 1) grid = 1;
+    // CTAs: a multiple of the slab count, at most two per SM, no more than there are row tiles
+    uint32_t per_slab = (2u * dev.sms) / a.slabs;
+    if (per_slab > a.row_tiles) per_slab = a.row_tiles;
+    if (per_slab < 1) per_slab = 1;
+    const int grid = static_cast<int>(per_slab * a.slabs);
     return weight ? run_quant<true>(b, map, a, grid, st) : run_quant<false>(b, map, a, grid, st);
 }
 
@@ -238,10 +267,12 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
                       kBKBytes, BN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MACAQ_OK) return s;
 
+    // persistent: at most one CTA per SM; the CTAs walk the tiles (grouped: the tile count is
+    // only known on the device, so the bound uses ceil(rows/128) + E row tiles)
     const int64_t m_tiles = grouped ? (rows + 127) / 128 + experts : (rows + 127) / 128;
-    if (m_tiles > 65535) return MACAQ_ERR_SHAPE;
-    dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(m_tiles));
-    if (BN == 256) return grouped ? run_gemm<256, true>(amap, bmap, g, grid, st) : run_gemm<256, false>(amap, bmap, g, grid, st);
+    const int64_t tiles = m_tiles * (N / BN);
+    const unsigned grid = static_cast<unsigned>(tiles < dev.sms ? tiles : dev.sms);
+    if (BN == 256) return grouped ? run_gemm<256, true>(amap, bmap, g, dim3(grid), st) : run_gemm<256, false>(amap, bmap, g, dim3(grid), st);
     return grouped ? run_gemm<128, true>(amap, bmap, g, grid, st) : run_gemm<128, false>(amap, bmap, g, grid, st);
 }
 

@@ -9,12 +9,12 @@
 //   code = E2M1_rne_satfinite(v[k] * 2^(127-E)), two codes per byte, even k in the low nibble
 // Sources: aipolix.com page on MACaQ (Persian), paragraphs 2-3; OCP Microscaling Formats v1.0.
 //
-// Data movement: the bf16 input is viewed as a flat array of 128-byte lines and streamed through
-// shared memory by TMA (16 KB tiles = 256 groups, 128-byte swizzle so that each thread's 64-byte
-// group is read without bank conflicts), in a 4-stage mbarrier ring per CTA; one thread owns one
-// group, so the Hadamard stages up to b = 32 stay in registers and b = 64 / 128 add one / two
-// shuffle stages with the neighbouring lanes. Codes go out as one 16-byte store per group; four
-// neighbouring lanes combine their E8M0 bytes into one 32-bit store in the tiled SF layout.
+// Data movement: the bf16 input is cut into tiles of (256 / w) rows x w groups (w = 32, 16, 8 or 4
+// groups, the largest that divides K/32), always 16 KB, streamed through shared memory by TMA with
+// the 128-byte swizzle (each thread's 64-byte group is read without bank conflicts). One thread owns
+// one group; the Hadamard stages up to b = 32 stay in registers (packed fp32 pairs), b = 64 / 128 add
+// one / two shuffle stages with the neighbouring lanes. Codes go out as one 16-byte store per group;
+// four neighbouring lanes combine their E8M0 bytes into one 32-bit store in the tiled SF layout.
 #pragma once
 
 #include "groups.cuh"
@@ -22,10 +22,10 @@
 
 namespace macaq {
 
-constexpr int kQThreads = 256;
-constexpr int kQGroupsPerTile = 256;                 // one group per thread
-constexpr int kQTileBytes = kQGroupsPerTile * 64;    // 16 KB of bf16
-constexpr int kQTileLines = kQTileBytes / 128;       // 128-byte lines per tile (TMA box height)
+constexpr int kQConsumerWarps = 8;
+constexpr int kQConsumers = kQConsumerWarps * 32;    // one 32-element group per consumer thread per tile
+constexpr int kQThreads = kQConsumers + 32;          // + one producer warp
+constexpr int kQTileBytes = kQConsumers * 64;        // 16 KB of bf16
 constexpr int kQStages = 4;
 
 struct QuantArgs {
@@ -36,9 +36,12 @@ struct QuantArgs {
     float *inv_s;             // weights: receives 1/mul (IEEE division), or nullptr
     int64_t rows;
     uint32_t K;
-    uint32_t kg;              // K / 32
-    uint32_t total_groups;    // rows * K / 32
-    uint32_t num_tiles;
+    uint32_t kg;              // K / 32 groups per row
+    uint32_t slab_groups;     // groups per column slab: 32, 16, 8 or 4 (divides kg)
+    uint32_t slab_shift;      // log2(slab_groups)
+    uint32_t slabs;           // kg / slab_groups
+    uint32_t tile_rows;       // rows per tile = 256 / slab_groups
+    uint32_t row_tiles;       // ceil(rows / tile_rows)
     int32_t E;                // groups (experts); 1 for a dense call
     uint64_t wait_limit_ns;
 };
@@ -47,175 +50,208 @@ __host__ __device__ constexpr size_t quant_smem_bytes(int E) {
     return 1024 + static_cast<size_t>(kQStages) * kQTileBytes + 2 * sizeof(int32_t) * (E + 1);
 }
 
+// The 32 values of a group live in 16 packed pairs p[i] = (v[2i], v[2i+1]).
+// Butterfly stage h = 1 pairs the two lanes of one register; stages h >= 2 pair register i with
+// register i + h/2 lane by lane, so they run as packed adds/subtracts.
 template <int kB>
-__device__ __forceinline__ void fwht_in_thread(float (&x)[32]) {
-    constexpr int kLim = kB < 32 ? kB : 32;
+__device__ __forceinline__ void fwht_in_thread(uint64_t (&p)[16]) {
+    if constexpr (kB >= 2) {
 #pragma unroll
-    for (int h = 1; h < kLim; h <<= 1) {
+        for (int i = 0; i < 16; ++i) {
+            float a, c;
+            upk2(p[i], a, c);
+            p[i] = pk2(__fadd_rn(a, c), __fsub_rn(a, c));
+        }
+    }
+    constexpr int kLim = (kB < 32 ? kB : 32) / 2;  // stages h = 2 .. min(b, 32)/2, as h/2
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            if ((j & h) == 0) {
-                const float u = x[j], w = x[j + h];
-                x[j] = __fadd_rn(u, w);
-                x[j + h] = __fsub_rn(u, w);
+    for (int hp = 1; hp < kLim; hp <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if ((i & hp) == 0) {
+                const uint64_t a = p[i], c = p[i + hp];
+                p[i] = add2(a, c);
+                p[i + hp] = sub2(a, c);
             }
         }
     }
 }
 
-// One cross-lane butterfly stage: this lane's group is paired with lane ^ lane_bit's group.
-__device__ __forceinline__ void fwht_cross_lane(float (&x)[32], int lane_bit) {
+// One cross-lane butterfly stage: this lane's group is paired with lane ^ lane_bit's group
+// (the next group of the same row).
+__device__ __forceinline__ void fwht_cross_lane(uint64_t (&p)[16], int lane_bit) {
     const bool upper = (threadIdx.x & lane_bit) != 0;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float o = __shfl_xor_sync(0xffffffffu, x[j], lane_bit);
-        x[j] = upper ? __fsub_rn(o, x[j]) : __fadd_rn(x[j], o);
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, p[i], lane_bit);
+        p[i] = upper ? sub2(o, p[i]) : add2(p[i], o);
     }
 }
 
+__device__ __forceinline__ void load_mul(const float *mul, uint64_t (&mv)[16]) {
+    const float4 *mp = reinterpret_cast<const float4 *>(mul);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 f = __ldg(mp + i);
+        mv[2 * i] = pk2(f.x, f.y);
+        mv[2 * i + 1] = pk2(f.z, f.w);
+    }
+}
+
+// Work split: the K axis is cut into column slabs of slab_groups groups; a tile is tile_rows rows of
+// one slab (always 256 groups, 16 KB). A CTA keeps one slab for its whole life and walks its row
+// tiles, so each consumer thread owns one fixed group column and keeps that column's 32 multipliers
+// in registers. A producer warp streams the tiles with TMA (3-D tensor map rows x 128-byte chunks x
+// 64 elements, 128-byte swizzle) into a 4-stage ring with full/empty mbarriers.
 template <int kB, bool kWeight>
-__global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a) {
+__global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a) {
     extern __shared__ uint8_t dsmem[];
     __shared__ uint64_t full_bar[kQStages];
+    __shared__ uint64_t empty_bar[kQStages];
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     int32_t *s_off = reinterpret_cast<int32_t *>(tiles + kQStages * kQTileBytes);
     int32_t *s_tb = s_off + (a.E + 1);
 
     const int tid = threadIdx.x;
+    const int warp = tid >> 5;
     const int lane = tid & 31;
+    const uint32_t slab = blockIdx.x % a.slabs;
+    const uint32_t ctas_per_slab = gridDim.x / a.slabs;
+    const uint32_t first_tile = blockIdx.x / a.slabs;
 
     if (tid == 0) {
-        for (int s = 0; s < kQStages; ++s) mbar_init(&full_bar[s], 1);
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kQConsumerWarps);
+        }
         fence_mbar_init();
-        if (a.num_tiles > 0) prefetch_tensor_map(&xmap);
+        if (first_tile < a.row_tiles) prefetch_tensor_map(&xmap);
     }
     load_group_layout(a.offsets, a.E, a.rows, s_off, s_tb);  // contains __syncthreads
 
-    // prologue: the first kQStages-1 tiles of this CTA
-    if (tid == 0) {
-        for (int s = 0; s < kQStages - 1; ++s) {
-            const uint32_t t = blockIdx.x + s * gridDim.x;
-            if (t < a.num_tiles) {
+    if (warp == kQConsumerWarps) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            uint32_t j = 0;
+            for (uint32_t rt = first_tile; rt < a.row_tiles; rt += ctas_per_slab, ++j) {
+                const int s = j % kQStages;
+                if (j >= kQStages && !mbar_wait(&empty_bar[s], ((j / kQStages) & 1) ^ 1, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&full_bar[s], kQTileBytes);
-                tma_load_2d(tiles + s * kQTileBytes, &xmap, &full_bar[s], 0, static_cast<int32_t>(t * kQTileLines));
+                tma_load_3d(tiles + s * kQTileBytes, &xmap, &full_bar[s], 0,
+                            static_cast<int32_t>(slab * (a.slab_groups / 2)), static_cast<int32_t>(rt * a.tile_rows));
+            }
+            // let the copies this thread issued land before the CTA can exit
+            for (uint32_t i = (j > kQStages ? j - kQStages : 0); i < j; ++i)
+                if (!mbar_wait(&full_bar[i % kQStages], (i / kQStages) & 1, 2000000000ull)) break;
+        }
+    } else {
+        // ---------------------------------------------------------------- consumers
+        const uint32_t gc = tid & (a.slab_groups - 1);      // group within the slab
+        const uint32_t r_in = tid >> a.slab_shift;          // row within the tile
+        const uint32_t g = slab * a.slab_groups + gc;       // group column of this thread
+        const uint32_t line = r_in * (a.slab_groups / 2) + (gc >> 1);  // 128-byte line of the tile
+        uint64_t mv[16];
+        int cur_e = -1;
+        uint32_t j = 0;
+        for (uint32_t rt = first_tile; rt < a.row_tiles; rt += ctas_per_slab, ++j) {
+            const int s = j % kQStages;
+            const uint32_t m = rt * a.tile_rows + r_in;
+            const bool valid = m < a.rows;
+            const int e = valid ? find_group(s_off, a.E, m) : -1;
+            if (a.mul != nullptr && e != cur_e && e >= 0) {   // per-channel multipliers of this column
+                load_mul(a.mul + static_cast<uint64_t>(e) * a.K + g * 32, mv);
+                cur_e = e;
+            }
+            // the whole warp leaves together if any lane's wait ran out (shuffles follow)
+            if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[s], (j / kQStages) & 1, a.wait_limit_ns))) break;
+
+            const uint8_t *lp = tiles + s * kQTileBytes + line * 128;
+            uint4 raw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int phys = (((gc & 1) << 2) + i) ^ (line & 7);
+                raw[i] = *reinterpret_cast<const uint4 *>(lp + phys * 16);
+            }
+            uint64_t p[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                p[4 * i + 0] = pk2(__uint_as_float(raw[i].x << 16), __uint_as_float(raw[i].x & 0xFFFF0000u));
+                p[4 * i + 1] = pk2(__uint_as_float(raw[i].y << 16), __uint_as_float(raw[i].y & 0xFFFF0000u));
+                p[4 * i + 2] = pk2(__uint_as_float(raw[i].z << 16), __uint_as_float(raw[i].z & 0xFFFF0000u));
+                p[4 * i + 3] = pk2(__uint_as_float(raw[i].w << 16), __uint_as_float(raw[i].w & 0xFFFF0000u));
+            }
+            // Release the stage only after every lane has its words in registers (the unpacking above
+            // consumed them), and order those generic-proxy reads before the next TMA write of the
+            // stage, which is an async-proxy access.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[s]);
+            if (a.mul != nullptr) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
+            }
+
+            if constexpr (kB > 1) {
+                fwht_in_thread<kB>(p);
+                if constexpr (kB >= 64) fwht_cross_lane(p, 1);
+                if constexpr (kB >= 128) fwht_cross_lane(p, 2);
+                if constexpr (kWeight) {
+                    const uint64_t inv_b = pk2(1.0f / kB, 1.0f / kB);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], inv_b);
+                }
+            }
+
+            float mx[16];  // max |v| as a tree: short dependency chains
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float lo, hi;
+                upk2(p[i], lo, hi);
+                mx[i] = fmaxf(fabsf(lo), fabsf(hi));
+            }
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+            const int ef = static_cast<int>(__float_as_uint(mx[0]) >> 23);  // biased exponent (amax >= 0)
+            const uint32_t E8 = static_cast<uint32_t>(ef > 2 ? ef - 2 : 0);
+            const float inv_scale = __uint_as_float((254u - E8) << 23);     // 2^(127 - E), a normal float
+            const uint64_t inv_scale2 = pk2(inv_scale, inv_scale);
+
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) upk2(mul2(p[i], inv_scale2), y[2 * i], y[2 * i + 1]);
+            uint4 packed;
+            packed.x = cvt_e2m1x8(y + 0);
+            packed.y = cvt_e2m1x8(y + 8);
+            packed.z = cvt_e2m1x8(y + 16);
+            packed.w = cvt_e2m1x8(y + 24);
+            const bool store = e >= 0;
+            if (store)
+                *reinterpret_cast<uint4 *>(a.q + static_cast<uint64_t>(m) * (a.K / 2) + g * 16) = packed;
+
+            // lanes 4i..4i+3 hold scale columns 4c..4c+3 of one row: one 32-bit store
+            const uint32_t b1 = __shfl_down_sync(0xffffffffu, E8, 1);
+            const uint32_t b2 = __shfl_down_sync(0xffffffffu, E8, 2);
+            const uint32_t b3 = __shfl_down_sync(0xffffffffu, E8, 3);
+            if (store && (lane & 3) == 0) {
+                const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + (m - static_cast<uint32_t>(s_off[e]));
+                *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, g, a.kg >> 2)) =
+                    E8 | (b1 << 8) | (b2 << 16) | (b3 << 24);
             }
         }
     }
 
-    uint32_t it = 0;
-    bool ok = true;
-    for (uint32_t t = blockIdx.x; t < a.num_tiles; t += gridDim.x, ++it) {
-        const int s = it % kQStages;
-        const bool ready = mbar_wait(&full_bar[s], (it / kQStages) & 1, a.wait_limit_ns);
-        // every thread is done with tile it-1 and tile it has landed
-        if (!__syncthreads_and(ready)) {
-            ok = false;
-            break;
-        }
-        if (tid == 0) {
-            const uint32_t tn = t + (kQStages - 1) * gridDim.x;
-            if (tn < a.num_tiles) {
-                const int sn = (it + kQStages - 1) % kQStages;  // the stage tile it-1 used
-                mbar_arrive_expect_tx(&full_bar[sn], kQTileBytes);
-                tma_load_2d(tiles + sn * kQTileBytes, &xmap, &full_bar[sn], 0, static_cast<int32_t>(tn * kQTileLines));
-            }
-        }
-
-        const uint32_t gi = t * kQGroupsPerTile + tid;  // global group index
-        const bool valid = gi < a.total_groups;
-        const uint32_t m = valid ? gi / a.kg : 0;
-        const uint32_t g = valid ? gi - m * a.kg : 0;
-        const int e = valid ? find_group(s_off, a.E, m) : -1;
-
-        // 64 bytes of this group from the swizzled tile: line tid/2, logical chunks (tid&1)*4 + i
-        const uint8_t *line = tiles + s * kQTileBytes + (tid >> 1) * 128;
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int phys = (((tid & 1) << 2) + i) ^ ((tid >> 1) & 7);
-            const uint4 v = *reinterpret_cast<const uint4 *>(line + phys * 16);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                x[8 * i + 2 * p] = __uint_as_float(w[p] << 16);
-                x[8 * i + 2 * p + 1] = __uint_as_float(w[p] & 0xFFFF0000u);
-            }
-        }
-
-        if (a.mul != nullptr) {
-            const int eg = e < 0 ? 0 : e;
-            const float4 *mp = reinterpret_cast<const float4 *>(a.mul + static_cast<uint64_t>(eg) * a.K + g * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 mv = __ldg(mp + i);
-                x[4 * i + 0] = __fmul_rn(x[4 * i + 0], mv.x);
-                x[4 * i + 1] = __fmul_rn(x[4 * i + 1], mv.y);
-                x[4 * i + 2] = __fmul_rn(x[4 * i + 2], mv.z);
-                x[4 * i + 3] = __fmul_rn(x[4 * i + 3], mv.w);
-            }
-        }
-
-        if constexpr (kB > 1) {
-            fwht_in_thread<kB>(x);
-            if constexpr (kB >= 64) fwht_cross_lane(x, 1);
-            if constexpr (kB >= 128) fwht_cross_lane(x, 2);
-            if constexpr (kWeight) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], 1.0f / kB);
-            }
-        }
-
-        float amax = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(x[j]));
-        const int ef = static_cast<int>(__float_as_uint(amax) >> 23);  // biased exponent (amax >= 0)
-        const uint32_t E8 = static_cast<uint32_t>(ef > 2 ? ef - 2 : 0);
-        const float inv_scale = __uint_as_float((254u - E8) << 23);   // 2^(127 - E), a normal float
-
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], inv_scale);
-        uint4 packed;
-        packed.x = cvt_e2m1x8(x + 0);
-        packed.y = cvt_e2m1x8(x + 8);
-        packed.z = cvt_e2m1x8(x + 16);
-        packed.w = cvt_e2m1x8(x + 24);
-        const bool store = valid && e >= 0;
-        if (store) *reinterpret_cast<uint4 *>(a.q + static_cast<uint64_t>(gi) * 16) = packed;
-
-        // lanes 4i..4i+3 hold scale columns 4c..4c+3 of one row: one 32-bit store
-        const uint32_t b1 = __shfl_down_sync(0xffffffffu, E8, 1);
-        const uint32_t b2 = __shfl_down_sync(0xffffffffu, E8, 2);
-        const uint32_t b3 = __shfl_down_sync(0xffffffffu, E8, 3);
-        if (store && (lane & 3) == 0) {
-            const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + (m - static_cast<uint32_t>(s_off[e]));
-            *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, g, a.kg >> 2)) =
-                E8 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        }
-    }
-
-    if (!ok) {
-        // a tile never arrived: wait (bounded) for the copies this CTA still has in flight
-        if (tid == 0) {
-            for (uint32_t j = it; j < it + kQStages - 1; ++j) {
-                const uint32_t tj = blockIdx.x + j * gridDim.x;
-                if (tj >= a.num_tiles) break;
-                if (!mbar_wait(&full_bar[j % kQStages], (j / kQStages) & 1, 2000000000ull)) break;
-            }
-        }
-        return;
-    }
-
-    // zero the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1)
+    // zero the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1):
+    // one warp per padding row, lanes over the 32-bit words (4 scale columns each) of that row
     const uint32_t kq = a.kg >> 2;
     for (int e = blockIdx.x; e < a.E; e += gridDim.x) {
         const uint32_t me = static_cast<uint32_t>(s_off[e + 1] - s_off[e]);
         const uint32_t nt = static_cast<uint32_t>(s_tb[e + 1] - s_tb[e]);
-        const uint32_t words = (nt * 128 - me) * kq;
-        for (uint32_t w = tid; w < words; w += blockDim.x) {
-            const uint32_t pr = me + w / kq;
-            const uint32_t c4 = (w - (w / kq) * kq) * 4;
+        for (uint32_t pr = me + warp; pr < nt * 128; pr += kQThreads / 32) {
             const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + pr;
-            *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, c4, kq)) = 0u;
+            for (uint32_t w = lane; w < kq; w += 32)
+                *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, 4 * w, kq)) = 0u;
         }
     }
 
