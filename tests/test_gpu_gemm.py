@@ -64,6 +64,7 @@ def check_dense(Aq, Asf, Wq, Wsf, rows=None):
 @pytest.mark.parametrize("M,N,K", [
     (16, 256, 256), (1, 128, 128), (3, 384, 384), (17, 256, 768), (128, 256, 512),
     (129, 512, 512), (300, 128, 1024), (256, 768, 4096), (64, 1024, 5120),
+    (300, 256, 384), (513, 512, 1280), (1024, 1024, 2048),
 ])
 def test_random_codes(M, N, K):
     check_dense(*random_operands(M * 7 + N + K, M, N, K))

@@ -4,11 +4,12 @@
 //
 // fp32 accumulation in tensor memory, bf16 (round-to-nearest-even) or fp32 output. Dense and grouped
 // (MoE) forms; the grouped form maps each 128-row tile to its expert from the device-side offsets.
+// gemm_mxf4_pair_kernel is the dense form on 2-SM pairs (cta_group::2, 256-row tiles).
 // Source: glonce.com page on MACaQ, paragraph 5 (W4A4 dense and grouped matmul kernels).
 //
 // Persistent kernel: one CTA per SM walks output tiles of 128 x BN (BN = 256, or 128 when
 // N % 256 != 0) in a grouped raster (bands of kRasterM row tiles) so that the operands of the tiles
-// in flight stay in L2. Warp roles (192 threads):
+// in flight stay in L2. Warp roles (320 threads):
 //   warp 0      TMA producer: per K-block of 256 elements, the A tile (128 rows x 128 bytes) and the
 //               B tile (BN rows x 128 bytes) with 128-byte swizzle via tensor maps, plus the matching
 //               scale-factor tiles (already in the tcgen05 128x4 tiling) by plain bulk copies. It runs
@@ -17,9 +18,10 @@
 //               then per K-block copies the scale factors into TMEM (tcgen05.cp 32x128b.warpx4),
 //               issues 4 MMAs of 128 x BN x 64 and frees the stage with tcgen05.commit; a final commit
 //               per tile signals the epilogue.
-//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator (each warp reads its 32-lane quarter);
-//               for bf16 output the whole row is pulled into registers and the accumulator released
-//               before the global stores, so the next tile's MMAs overlap the stores.
+//   warps 2-9   epilogue: tcgen05.ld of the fp32 accumulator (each warp reads its 32-lane quarter
+//               and one half of the columns); for bf16 output the values are pulled into registers
+//               and the accumulator released before the global stores, so the next tile's MMAs
+//               overlap the stores.
 // Every wait is bounded; a timeout anywhere stops all roles of the CTA, lets its own copies and
 // MMAs land, frees TMEM and returns.
 #pragma once
@@ -33,7 +35,8 @@ namespace macaq {
 
 constexpr int kBM = 128;
 constexpr int kBKBytes = 128;  // 256 FP4 elements per K-block
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;   // producer warp, MMA warp, 8 epilogue warps
+constexpr int kEpiWarps = 8;
 constexpr int kRasterM = 16;   // row tiles per raster band
 constexpr uint64_t kDrainLimitNs = 2000000000ull;  // waits for the kernel's own copies / MMAs to land
 
@@ -99,6 +102,62 @@ __device__ __forceinline__ void raster(uint32_t t, uint32_t m_tiles, uint32_t n_
     nt = r / height;
 }
 
+// Epilogue of one output tile for one epilogue warp. Warp w (2..9) reads TMEM lane quarter w % 4
+// (rows quarter*32 .. +31 of the CTA's 128) and column half (w - 2) / 4 of the BN columns. For bf16
+// output the warp's 32 x BN/2 block is pulled into registers and the accumulator released (one
+// arrival per warp on accum_empty, possibly in the leader CTA of a pair) before the global stores,
+// so the next tile's MMAs overlap them; fp32 output keeps TMEM until its stores are issued.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(uint32_t tmem, int warp, int lane, int64_t row0, int64_t row_end,
+                                              int64_t col0, const GemmArgs &g, uint32_t accum_empty_addr) {
+    constexpr int kCols = BN / 2;  // columns per warp
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * kCols;
+    const int64_t row = row0 + quarter * 32 + lane;
+    const bool live = row < row_end;
+    const int64_t c0 = col0 + half * kCols;
+    if (g.out_f32) {
+#pragma unroll 1
+        for (int cb = 0; cb < kCols / 64; ++cb) {
+            uint32_t v[64];
+            tmem_ld64(taddr + cb * 64, v);
+            tmem_ld_wait();
+            if (!live) continue;
+            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(g.y) + row * g.N + c0 + cb * 64);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+    } else {
+        uint32_t packed[kCols / 2];
+#pragma unroll
+        for (int cb = 0; cb < kCols / 64; ++cb) {
+            uint32_t v[64];
+            tmem_ld64(taddr + cb * 64, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                packed[cb * 32 + k] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+        if (live) {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(g.y) + row * g.N + c0);
+#pragma unroll
+            for (int i = 0; i < kCols / 8; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+    }
+}
+
 template <int BN, bool kGrouped>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, GemmArgs g) {
@@ -135,7 +194,7 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&accum_full, 1);
-        mbar_init(&accum_empty, 4);  // one arrival per epilogue warp
+        mbar_init(&accum_empty, kEpiWarps);  // one arrival per epilogue warp
         failed = 0;
         fence_mbar_init();
         prefetch_tensor_map(&amap);
@@ -265,9 +324,7 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
         }
     } else {
         // ---------------------------------------------------------------- epilogue
-        const int quarter = warp & 3;  // TMEM lanes this warp may read
-        const int r = quarter * 32 + lane;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t empty_addr = smem_u32(&accum_empty);
         uint32_t tiles_done = 0;
         for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tiles_done) {
             uint32_t mt, nt;
@@ -278,50 +335,7 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
             if (!mbar_wait_or_abort(&accum_full, tiles_done & 1, limit, &failed)) break;
             tc_fence_after();
             if (failed) break;
-            const int64_t row = row0 + r;
-            const bool live = row < row_end;
-            const int64_t col0 = static_cast<int64_t>(nt) * BN;
-            if (g.out_f32) {
-                // fp32 (checking) output: read and store 32 columns at a time, then release TMEM
-#pragma unroll 1
-                for (int cb = 0; cb < BN / 32; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + cb * 32, v);
-                    tmem_ld_wait();
-                    if (!live) continue;
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(g.y) + row * g.N + col0 + cb * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accum_empty);
-            } else {
-                // bf16 output: pull the whole row into registers, release TMEM, then store
-                uint32_t packed[BN / 2];
-#pragma unroll
-                for (int cb = 0; cb < BN / 32; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + cb * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-                        packed[cb * 16 + k] = *reinterpret_cast<uint32_t *>(&b2);
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accum_empty);
-                if (live) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(g.y) + row * g.N + col0);
-#pragma unroll
-                    for (int i = 0; i < BN / 8; ++i)
-                        dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-                }
-            }
+            epilogue_tile<BN>(tmem, warp, lane, row0, row_end, static_cast<int64_t>(nt) * BN, g, empty_addr);
         }
     }
 
@@ -329,6 +343,211 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ============================================================================ 2-SM pairs
+// Dense GEMM on clusters of two CTAs (cta_group::2): a pair computes a 256 x 256 output tile. CTA r
+// of the pair loads its 128 rows of A and rows [128r, 128r + 128) of the tile's 256 rows of B; the
+// even CTA (the leader) issues the 256 x 256 x 64 MMAs, which read A and B from both CTAs' shared
+// memory and leave each CTA's 128 rows of the accumulator in its own TMEM. Each CTA moves A + B/2
+// per K-block instead of A + B.
+//
+// Scale factors: the MMA reads them from TMEM, four-fold replicated over the lane quarters. Six
+// 32x128b.warpx4 copies per K-block (each about as costly as a whole 4 KB copy, together longer
+// than the K-block's MMAs) are replaced by three 128x256b copies, whose source must hold the four
+// replicas. TMA builds that source directly: a 4-D view of the tiled SF buffer, (128 bytes, tile
+// half h, 8-row group i, 128x4 tile c) with strides (h: next tile, i: 128 B, c: 512 B), turns one
+// 1 KB box into one replica laid out as [i][h][128 B]; four boxes give the 4 KB source of one copy.
+// This path needs K % 256 == 0 (the K-block's two 128x4 tiles sit next to each other).
+//
+// Synchronisation: all TMA loads of both CTAs complete on the leader's full barrier (the leader
+// expects both CTAs' bytes); the leader's commit frees the stage in both CTAs (multicast); the
+// per-tile accumulator signals go to both CTAs; every epilogue warp of both CTAs releases the
+// accumulator on the leader's accum_empty barrier.
+struct PairCfg {
+    static constexpr int kStages = 5;
+    static constexpr int kABytes = 128 * kBKBytes;      // this CTA's 128 rows of A
+    static constexpr int kBBytes = 128 * kBKBytes;      // this CTA's half of the 256 B rows
+    static constexpr int kSfxBytes = 12288;             // replicated SF: A 4 KB, then B 4 KB per chunk
+    static constexpr int kStageBytes = kABytes + kBBytes + kSfxBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
+    static constexpr int kTmemSfa = 256;
+    static constexpr int kTmemSfb = 264;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kThreads = kGemmThreads + 32;  // + a second producer warp for the scale factors
+};
+
+__global__ void __launch_bounds__(PairCfg::kThreads, 1)
+gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                      const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
+                      GemmArgs g, int sf_replica_boxes) {
+    using C = PairCfg;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t dsmem[];
+    __shared__ uint64_t full_bar[S];
+    __shared__ uint64_t empty_bar[S];
+    __shared__ uint64_t accum_full;
+    __shared__ uint64_t accum_empty;   // used in the leader: 16 arrivals (8 warps x 2 CTAs) per tile
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int failed;
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + S * C::kABytes;
+    uint8_t *sSfx = sB + S * C::kBBytes;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const uint32_t cluster = blockIdx.x >> 1;
+    const uint32_t clusters = gridDim.x >> 1;
+    const uint32_t m_tiles = static_cast<uint32_t>((g.rows + 255) / 256);
+    const uint32_t n_tiles = static_cast<uint32_t>(g.N / 256);
+    const uint32_t num_tiles = m_tiles * n_tiles;  // the host launches at most this many pairs
+    const int K = g.K;
+    const int kq = K / 128;
+    const int num_kb = K / 256;
+    const uint64_t limit = g.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&accum_full, 1);
+        mbar_init(&accum_empty, 2 * kEpiWarps);
+        // (the leader's full barrier: one expect-tx arrival; both producer warps' copies complete it)
+        failed = 0;
+        fence_mbar_init();
+        prefetch_tensor_map(&amap);
+        prefetch_tensor_map(&bmap);
+        prefetch_tensor_map(&sfamap);
+        prefetch_tensor_map(&sfbmap);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_slot, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint32_t leader_failed_addr = map_to_rank(smem_u32(const_cast<int *>(&failed)), 0);
+
+    if (warp == 0 || warp == 10) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ TMA producers (both CTAs)
+            // warp 0: A and B (and the expect-tx of both CTAs' bytes); warp 10: the scale factors
+            const bool sf = warp == 10;
+            uint32_t j = 0;
+            bool stop = false;
+            for (uint32_t t = cluster; t < num_tiles && !stop; t += clusters) {
+                uint32_t mt, nt;
+                raster(t, m_tiles, n_tiles, mt, nt);
+                const int32_t arow = static_cast<int32_t>(mt * 256 + rank * 128);
+                const int32_t brow = static_cast<int32_t>(nt * 256 + rank * 128);
+                const int32_t a_tile = static_cast<int32_t>((mt * 2 + rank) * kq);   // first 128x4 tile of A's rows
+                const int32_t b_tile = static_cast<int32_t>(nt * 2 * kq);            // of B's first 128 rows
+                for (int kb = 0; kb < num_kb; ++kb, ++j) {
+                    const int s = j % S;
+                    if (j >= S && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) {
+                        stop = true;
+                        break;
+                    }
+                    if (!sf) {
+                        if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * C::kStageBytes);
+                        tma_load_2d_pair(sA + s * C::kABytes, &amap, &full_bar[s], kb * kBKBytes, arow);
+                        tma_load_2d_pair(sB + s * C::kBBytes, &bmap, &full_bar[s], kb * kBKBytes, brow);
+                    } else {
+                        // four replicas each: A (halves = the K-block's tiles), B chunk 0, 1 (halves = rows)
+                        uint8_t *x = sSfx + s * C::kSfxBytes;
+                        if (sf_replica_boxes == 1) {
+                            tma_load_5d_pair(x, &sfamap, &full_bar[s], 0, 0, 0, 0, a_tile + 2 * kb);
+                            tma_load_5d_pair(x + 4096, &sfbmap, &full_bar[s], 0, 0, 0, 0, b_tile + 2 * kb);
+                            tma_load_5d_pair(x + 8192, &sfbmap, &full_bar[s], 0, 0, 0, 0, b_tile + 2 * kb + 1);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                tma_load_4d_pair(x + q * 1024, &sfamap, &full_bar[s], 0, 0, 0, a_tile + 2 * kb);
+                                tma_load_4d_pair(x + 4096 + q * 1024, &sfbmap, &full_bar[s], 0, 0, 0, b_tile + 2 * kb);
+                                tma_load_4d_pair(x + 8192 + q * 1024, &sfbmap, &full_bar[s], 0, 0, 0, b_tile + 2 * kb + 1);
+                            }
+                        }
+                    }
+                }
+            }
+            // the leader's full barriers count both CTAs' bytes: let every issued copy land
+            if (leader && !sf)
+                for (uint32_t i = (j > S ? j - S : 0); i < j; ++i)
+                    if (!mbar_wait(&full_bar[i % S], (i / S) & 1, kDrainLimitNs)) break;
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------------------ MMA issuer (leader only)
+            const uint32_t idesc_lo = idesc_mxf4_m(256, 256, 0);
+            const uint32_t idesc_hi = idesc_mxf4_m(256, 256, 2);
+            uint32_t j = 0;
+            uint32_t tiles_done = 0;
+            bool stop = false;
+            for (uint32_t t = cluster; t < num_tiles && !stop; t += clusters, ++tiles_done) {
+                if (tiles_done > 0 && !mbar_wait_or_abort(&accum_empty, (tiles_done - 1) & 1, limit, &failed)) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < num_kb; ++kb, ++j) {
+                    const int s = j % S;
+                    if (!mbar_wait_or_abort(&full_bar[s], (j / S) & 1, limit, &failed)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfx = smem_u32(sSfx + s * C::kSfxBytes);
+                    tc_cp_sf_wide_pair(tmem + C::kTmemSfa, sdesc_sf_wide(sfx));
+                    tc_cp_sf_wide_pair(tmem + C::kTmemSfb, sdesc_sf_wide(sfx + 4096));
+                    tc_cp_sf_wide_pair(tmem + C::kTmemSfb + 8, sdesc_sf_wide(sfx + 8192));
+                    const uint64_t adesc = sdesc_sw128(smem_u32(sA + s * C::kABytes));
+                    const uint64_t bdesc = sdesc_sw128(smem_u32(sB + s * C::kBBytes));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c = q >> 1;
+                        tc_mma_mxf4_pair(tmem, adesc + 2 * q, bdesc + 2 * q, (q & 1) ? idesc_hi : idesc_lo,
+                                         tmem + C::kTmemSfa + 4 * c, tmem + C::kTmemSfb + c * 8, (kb | q) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair(&empty_bar[s]);
+                }
+                tc_commit_pair(&accum_full);
+            }
+            if (stop) {
+                tc_commit_pair(&accum_full);
+                ++tiles_done;
+            }
+            if (tiles_done > 0) mbar_wait(&accum_full, (tiles_done - 1) & 1, kDrainLimitNs);
+        }
+    } else if (warp >= 2 && warp < 10) {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const uint32_t empty_addr = map_to_rank(smem_u32(&accum_empty), 0);
+        uint32_t tiles_done = 0;
+        for (uint32_t t = cluster; t < num_tiles; t += clusters, ++tiles_done) {
+            uint32_t mt, nt;
+            raster(t, m_tiles, n_tiles, mt, nt);
+            if (!mbar_wait_or_abort(&accum_full, tiles_done & 1, limit, &failed)) break;
+            tc_fence_after();
+            int leader_failed;
+            asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(leader_failed) : "r"(leader_failed_addr) : "memory");
+            if (failed || leader_failed) break;
+            const int64_t row0 = static_cast<int64_t>(mt) * 256 + rank * 128;
+            const int64_t row_end = row0 + 128 < g.rows ? row0 + 128 : g.rows;
+            epilogue_tile<256>(tmem, warp, lane, row0, row_end, static_cast<int64_t>(nt) * 256, g, empty_addr);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its partner may still touch its barriers or shared memory
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, C::kTmemCols);
 }
 
 }  // namespace macaq

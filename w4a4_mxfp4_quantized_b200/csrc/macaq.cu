@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <array>
 #include <atomic>
 #include <cstring>
 #include <map>
@@ -75,12 +76,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-using MapKey = std::tuple<int, uintptr_t, int, int, uint64_t, uint64_t, uint64_t, uint64_t, uint64_t, uint32_t,
-                          uint32_t, uint32_t, int>;
+using MapKey = std::tuple<int, uintptr_t, int, int, std::array<uint64_t, 5>, std::array<uint64_t, 4>,
+                          std::array<uint32_t, 5>, int>;
 
-// A tiled tensor map of rank 2 or 3 over a strided array: dims[0] contiguous elements, dims[1] and
-// dims[2] with byte strides strides[0] and strides[1]; box of box[0] x box[1] (x box[2]) elements;
-// zero fill out of bounds. Descriptors are cached by everything they encode.
+// A tiled tensor map of rank 2 to 5 over a strided array: dims[0] contiguous elements, dims[i] with
+// byte stride strides[i-1]; box of box[0] x ... elements; zero fill out of bounds. Descriptors are
+// cached by everything they encode.
 macaq_status tensor_map(CUtensorMap *out, const void *base, CUtensorMapDataType dtype, int rank,
                         const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
                         CUtensorMapSwizzle swizzle) {
@@ -88,9 +89,16 @@ macaq_status tensor_map(CUtensorMap *out, const void *base, CUtensorMapDataType 
     static std::map<MapKey, CUtensorMap> cache;
     int dev = 0;
     cudaGetDevice(&dev);
-    const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int>(dtype), rank, dims[0], dims[1],
-                     rank > 2 ? dims[2] : 0, strides[0], rank > 2 ? strides[1] : 0, box[0], box[1],
-                     rank > 2 ? box[2] : 0, static_cast<int>(swizzle)};
+    std::array<uint64_t, 5> kd{};
+    std::array<uint64_t, 4> ks{};
+    std::array<uint32_t, 5> kb{};
+    for (int i = 0; i < rank; ++i) {
+        kd[i] = dims[i];
+        kb[i] = box[i];
+        if (i > 0) ks[i - 1] = strides[i - 1];
+    }
+    const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int>(dtype), rank, kd, ks, kb,
+                     static_cast<int>(swizzle)};
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end()) {
@@ -100,10 +108,15 @@ macaq_status tensor_map(CUtensorMap *out, const void *base, CUtensorMapDataType 
     auto fn = encode_fn();
     if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
     CUtensorMap m;
-    cuuint64_t d[3] = {dims[0], dims[1], rank > 2 ? dims[2] : 1};
-    cuuint64_t s[2] = {strides[0], rank > 2 ? strides[1] : 0};
-    cuuint32_t b[3] = {box[0], box[1], rank > 2 ? box[2] : 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
+    cuuint64_t d[5];
+    cuuint64_t s[4];
+    cuuint32_t b[5];
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        if (i > 0) s[i - 1] = strides[i - 1];
+    }
     CUresult r = fn(&m, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d, s, b, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -245,6 +258,7 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
 
     const int BN = (N % 256 == 0) ? 256 : 128;
     const bool grouped = offsets != nullptr;
+    const bool pair = !grouped && BN == 256 && rows > 128 && K % 256 == 0;  // 2-SM pairs, 256 x 256 tiles
     const int32_t experts = grouped ? E : 1;
     GemmArgs g;
     g.asf = Asf;
@@ -258,6 +272,63 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
     g.out_f32 = out_dtype == MACAQ_OUT_F32;
     g.bsf_stride = macaq_sf_bytes(N, K);
     g.wait_limit_ns = g_wait_limit_ns.load();
+
+    if (pair) {
+        CUtensorMap amap, bmap, sfamap, sfbmap;
+        s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+        if (s == MACAQ_OK)
+            s = tensor_map_2d(&bmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+        // replica views of the SF buffers: (128 B, half h, 8-row group i, 128x4 tile c); for A the
+        // halves are the K-block's two tiles (512 B apart), for B the two 128-row tiles of the
+        // 256-row N tile (K/128 tiles apart)
+        const uint64_t kq = static_cast<uint64_t>(K / 128);
+        // one 4 KB box holding all four replicas needs a zero-stride replica dimension; if the driver
+        // refuses that view, four 1 KB boxes (one replica each) are used instead
+        int replica_boxes = 1;
+        if (s == MACAQ_OK) {
+            const uint64_t da[5] = {128, 2, 4, 4, macaq_sf_bytes(rows, K) / 512};
+            const uint64_t sa[4] = {512, 128, 0, 512};
+            const uint64_t db[5] = {128, 2, 4, 4, macaq_sf_bytes(N, K) / 512};
+            const uint64_t sb[4] = {kq * 512, 128, 0, 512};
+            const uint32_t box[5] = {128, 2, 4, 4, 1};
+            if (tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, da, sa, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK ||
+                tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, db, sb, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK) {
+                replica_boxes = 4;
+                const uint64_t da4[4] = {128, 2, 4, macaq_sf_bytes(rows, K) / 512};
+                const uint64_t sa4[3] = {512, 128, 512};
+                const uint64_t db4[4] = {128, 2, 4, macaq_sf_bytes(N, K) / 512};
+                const uint64_t sb4[3] = {kq * 512, 128, 512};
+                const uint32_t box4[4] = {128, 2, 4, 1};
+                s = tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, da4, sa4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
+                if (s == MACAQ_OK)
+                    s = tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, db4, sb4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
+            }
+        }
+        if (s != MACAQ_OK) return s;
+        const int64_t tiles = ((rows + 255) / 256) * (N / 256);
+        const int64_t max_pairs = dev.sms / 2;
+        const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
+        s = set_smem(gemm_mxf4_pair_kernel, PairCfg::kSmemBytes);
+        if (s != MACAQ_OK) return s;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * pairs);
+        cfg.blockDim = dim3(PairCfg::kThreads);
+        cfg.dynamicSmemBytes = PairCfg::kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_mxf4_pair_kernel, amap, bmap, sfamap, sfbmap, g, replica_boxes);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaGetLastError();
+        return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+    }
 
     CUtensorMap amap, bmap;
     s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, kBM,
