@@ -93,8 +93,15 @@ size_t macaq_sf_bytes(int64_t rows, int64_t K);
  * Every expert's rows start on a fresh 128-row tile, so at most E extra tiles are needed. */
 size_t macaq_grouped_sf_bytes(int64_t total_rows, int32_t E, int64_t K);
 
-/* Workspace bytes macaq_linear / macaq_grouped_linear need for these sizes (E = 0 for dense).
- * 0 means no workspace is needed and `workspace` may be NULL. */
+/* Workspace bytes macaq_linear can use for these sizes on the current device (E = 0 for dense).
+ * Dense calls with M <= 128 and K % 256 == 0 given a workspace of at least this size run the skinny
+ * kernel (weights in
+ * the MMA's 128-row slot, the unit space split evenly over all SMs, split tiles reduced through the
+ * workspace); without a workspace they run the general kernel. 0 means no workspace is used.
+ * Contract: the workspace must be all zero before its first use; every call leaves it zero again
+ * (per-tile counters reset themselves), so one buffer can serve any number of consecutive calls.
+ * Calls that may run at the same time on different streams need separate workspaces. After a call
+ * that reported MACAQ_ERR_TIMEOUT, zero the workspace again. */
 size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E);
 
 /*
@@ -142,7 +149,9 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
  *                               macaq_act_quant; Asf is ignored.
  *   Wq, Wsf    from macaq_prep_weights: u8 [N, K/2] and the tiled SF of N rows
  *   Y          device [M, N], bf16 or fp32 per out_dtype (written)
- *   workspace  device scratch of at least macaq_workspace_bytes(M, N, K, 0) bytes (NULL if 0)
+ *   workspace  NULL, or device scratch of at least macaq_workspace_bytes(M, N, K, 0) bytes under the
+ *              contract above (selects the skinny kernel for M <= 128 and K % 256 == 0; too small:
+ *              MACAQ_ERR_WORKSPACE)
  * Source: glonce.com page, paragraph 5 (W4A4 dense matmul).
  */
 macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M,
@@ -158,7 +167,7 @@ macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const
  *   group_offsets  device int32 [E + 1] (as for macaq_act_quant); 1 <= E <= 1024
  *   Wq             device u8 [E, N, K/2];  Wsf device u8 [E, macaq_sf_bytes(N, K)]
  *   Y              device [total_rows, N] (written; only rows of some expert are written)
- *   workspace      device scratch of macaq_workspace_bytes(total_rows, N, K, E) bytes (NULL if 0)
+ *   workspace      unused in this version (may be NULL)
  * Source: glonce.com page, paragraph 5 (W4A4 grouped matmul).
  */
 macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,

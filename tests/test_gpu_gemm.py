@@ -28,10 +28,10 @@ def random_operands(seed, M, N, K, E=None):
     return Aq, Asf, Wq, Wsf
 
 
-def run_linear(Aq, Asf_tiled, Wq, Wsf_tiled, M, N, out_dtype):
+def run_linear(Aq, Asf_tiled, Wq, Wsf_tiled, M, N, out_dtype, use_workspace=True):
     Y = Guarded(M * N * (4 if out_dtype == mq.OUT_F32 else 2),
                 dtype=torch.float32 if out_dtype == mq.OUT_F32 else torch.bfloat16, shape=(M, N))
-    mq.linear(Aq, Asf_tiled, Wq, Wsf_tiled, out_dtype=out_dtype, Y=Y.t)
+    mq.linear(Aq, Asf_tiled, Wq, Wsf_tiled, out_dtype=out_dtype, Y=Y.t, use_workspace=use_workspace)
     torch.cuda.synchronize()
     assert Y.intact(), "write outside Y"
     assert mq.device_status() == 0
@@ -48,14 +48,14 @@ def assert_close(y_gpu, Y, T, rows=None):
     assert bad.size == 0, f"{len(bad)} outputs off, worst rel {np.max(err / (T + 1e-30)):.3g} at {bad[:3].tolist()}"
 
 
-def check_dense(Aq, Asf, Wq, Wsf, rows=None):
+def check_dense(Aq, Asf, Wq, Wsf, rows=None, use_workspace=True):
     M, N, K = Aq.shape[0], Wq.shape[0], Aq.shape[1] * 2
     dA = torch.from_numpy(Aq).cuda()
     dW = torch.from_numpy(Wq).cuda()
     dAsf = torch.from_numpy(swizzle(Asf, K)).cuda()
     dWsf = torch.from_numpy(swizzle(Wsf, K)).cuda()
-    y32 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_F32)
-    y16 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_BF16)
+    y32 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_F32, use_workspace)
+    y16 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_BF16, use_workspace)
     Y, T = oracle.linear(Aq, Asf, Wq, Wsf, rows=rows)
     assert_close(y32, Y, T, rows)
     assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
@@ -68,6 +68,32 @@ def check_dense(Aq, Asf, Wq, Wsf, rows=None):
 ])
 def test_random_codes(M, N, K):
     check_dense(*random_operands(M * 7 + N + K, M, N, K))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (16, 256, 256), (77, 384, 1280), (128, 512, 2048)])
+def test_general_kernel_at_small_m(M, N, K):
+    """Without a workspace, small M runs the general (non-skinny) kernel: same results."""
+    check_dense(*random_operands(M * 5 + N + K, M, N, K), use_workspace=False)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 4096), (5, 1024, 5120), (16, 14336 // 4, 4096), (128, 512, 1024)])
+def test_skinny_split_tiles(M, N, K):
+    """Skinny kernel with tiles split over several CTAs (partial sums reduced through the workspace),
+    called repeatedly on one workspace: the per-tile counters must reset themselves."""
+    ops = random_operands(M * 3 + N + K, M, N, K)
+    for _ in range(3):
+        check_dense(*ops)
+    ws = mq._workspace(torch.device("cuda"), 0)
+    assert int(ws.count_nonzero()) == 0
+
+
+def test_skinny_shared_workspace_across_shapes():
+    """Calls of different shapes share one workspace, whose layout (counts, then partials) moves with
+    N: each call must leave it all-zero so that the next call's counters start at zero."""
+    for M, N, K in [(1, 7168, 4096), (1, 14336, 2048), (3, 256, 4096), (1, 14336, 4096), (16, 1024, 5120)]:
+        check_dense(*random_operands(M + N + K, M, N, K), rows=np.array([0, M - 1]))
+        ws = mq._workspace(torch.device("cuda"), 0)
+        assert int(ws.count_nonzero()) == 0, (M, N, K)
 
 
 def test_extreme_scales_and_codes():

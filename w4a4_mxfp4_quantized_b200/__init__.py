@@ -115,6 +115,20 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+_ws_cache: dict = {}
+
+
+def _workspace(dev, nbytes: int) -> torch.Tensor:
+    """A zero-initialised scratch buffer per device, grown on demand and reused across calls (the
+    kernels leave it zeroed). Calls that may overlap on different streams need their own buffers."""
+    key = torch.device(dev).index
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        _ws_cache[key] = buf
+    return buf
+
+
 def sf_bytes(rows: int, K: int) -> int:
     """Bytes of the tiled scale-factor buffer of `rows` rows of K elements."""
     return int(lib().macaq_sf_bytes(rows, K))
@@ -170,16 +184,19 @@ def _out(M, N, out_dtype, dev, Y):
 
 def linear(A: torch.Tensor, Asf: torch.Tensor | None, Wq: torch.Tensor, Wsf: torch.Tensor, *,
            mode: int = A_QUANTIZED, inv_s: torch.Tensor | None = None, had_block: int = 32,
-           out_dtype: int = OUT_BF16, Y=None, workspace=None):
-    """Dense W4A4 linear Y = dq(A) dq(W')^T (fp32 accumulate; bf16 or fp32 out)."""
+           out_dtype: int = OUT_BF16, Y=None, workspace=None, use_workspace: bool = True):
+    """Dense W4A4 linear Y = dq(A) dq(W')^T (fp32 accumulate; bf16 or fp32 out).
+
+    With few rows (M <= 128) a workspace selects the skinny kernel (weights in the MMA's M slot,
+    split over all SMs); use_workspace=False runs the general kernel instead."""
     N = Wq.shape[0]
     K = Wq.shape[1] * 2
     M = A.shape[0]
     dev = A.device
     Y = _out(M, N, out_dtype, dev, Y)
-    ws_need = workspace_bytes(M, N, K, 0)
+    ws_need = workspace_bytes(M, N, K, 0) if use_workspace else 0
     if workspace is None and ws_need > 0:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+        workspace = _workspace(dev, ws_need)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("macaq_linear", lib().macaq_linear(
         mode, _ptr(A), _ptr(Asf), _ptr(inv_s), M, N, K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype,

@@ -550,4 +550,267 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     if (warp == 1) tmem_dealloc_pair(tmem, C::kTmemCols);
 }
 
+// ============================================================================ skinny (small M)
+// Dense GEMM for few rows (M <= 128, e.g. decode): the layer is a stream over W', so the weights take
+// the MMA's 128-row M slot and the M activation rows (padded to Mp, a multiple of 16) take its N
+// slot: D^T[n, m] = sum_k W'[n, k] X'[m, k]. The flattened space of (128-row W tile, K-block) units is
+// cut into equal contiguous ranges, one per CTA (one CTA per SM), so every SM streams the same number
+// of bytes. A CTA's range covers pieces of one or more tiles; a tile covered by one CTA is written
+// straight to Y (bf16 through shared memory and a TMA store), otherwise each piece's fp32 partial goes
+// to the workspace and the CTA that completes the tile's last piece (an atomic count per tile) adds
+// the pieces in their fixed order, writes Y and sets the partials and the count back to zero, so the
+// workspace is all-zero between calls whatever the shapes of earlier calls. When splitting tiles
+// would move more partial bytes than it saves (large M), the ranges are cut on whole tiles instead.
+// Both operands' scale factors arrive replicated (zero-stride TMA view) and go to TMEM with one wide
+// 128x256b copy each per K-block. The stage ring is as deep as shared memory allows; the accumulator
+// is double-buffered in TMEM. Needs K % 256 == 0.
+constexpr int kSkinnyMaxStages = 12;
+
+struct SkinnyArgs {
+    void *y;                   // [M, N]
+    float *partials;           // [tiles][max_pieces][M][128] fp32
+    int32_t *counts;           // [tiles], zero between calls
+    int32_t M, N, K;
+    int32_t mp;                // M rounded up to 16: the MMA's N
+    int32_t out_f32;
+    int32_t stages;
+    int32_t max_pieces;
+    uint32_t units;            // (N / 128) * (K / 256)
+    uint32_t gran;             // units per indivisible chunk: 1 (split tiles) or K-blocks per tile (whole tiles)
+    uint64_t wait_limit_ns;
+};
+
+__host__ __device__ constexpr int skinny_stage_bytes(int mp) { return 128 * kBKBytes + mp * kBKBytes + 8192; }
+__host__ __device__ constexpr int skinny_stage_bytes_y(int mp) { return mp * 128 * 2; }  // bf16 staging of one tile
+
+__global__ void __launch_bounds__(192, 1)
+gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
+                        const __grid_constant__ CUtensorMap sfwmap, const __grid_constant__ CUtensorMap sfxmap,
+                        const __grid_constant__ CUtensorMap ymap, SkinnyArgs g) {
+    extern __shared__ uint8_t dsmem[];
+    __shared__ uint64_t full_bar[kSkinnyMaxStages];
+    __shared__ uint64_t empty_bar[kSkinnyMaxStages];
+    __shared__ uint64_t accum_full[2];
+    __shared__ uint64_t accum_empty[2];
+    __shared__ uint64_t mma_done;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int32_t s_last;
+    __shared__ volatile int failed;
+
+    const int S = g.stages;
+    const int mp = g.mp;
+    const int stage_bytes = skinny_stage_bytes(mp);
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    uint8_t *sY = smem + S * stage_bytes;  // [4 warps][mp rows][32 columns] bf16
+    auto sW = [&](int s) { return smem + s * stage_bytes; };
+    auto sX = [&](int s) { return smem + s * stage_bytes + 128 * kBKBytes; };
+    auto sSfw = [&](int s) { return smem + s * stage_bytes + (128 + mp) * kBKBytes; };
+    auto sSfx = [&](int s) { return smem + s * stage_bytes + (128 + mp) * kBKBytes + 4096; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int K = g.K;
+    const int kq = K / 128;
+    const uint32_t num_kb = static_cast<uint32_t>(K / 256);
+    const uint32_t C = gridDim.x;
+    const uint32_t chunks = g.units / g.gran;  // ranges are cut on chunk boundaries
+    const uint32_t u_begin = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x) * chunks) / C) * g.gran;
+    const uint32_t u_end = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x + 1) * chunks) / C) * g.gran;
+    const uint64_t limit = g.wait_limit_ns;
+    // CTA covering unit u (the ranges above): largest c with floor(c * chunks / C) <= u / gran
+    auto cta_of = [&](uint32_t u) {
+        return static_cast<uint32_t>(((static_cast<uint64_t>(u / g.gran) + 1) * C - 1) / chunks);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accum_full[b], 1);
+            mbar_init(&accum_empty[b], 4);
+        }
+        mbar_init(&mma_done, 1);
+        failed = 0;
+        fence_mbar_init();
+        prefetch_tensor_map(&wmap);
+        prefetch_tensor_map(&xmap);
+        prefetch_tensor_map(&sfwmap);
+        prefetch_tensor_map(&sfxmap);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;                 // accumulators at columns 0 and 128
+    const uint32_t t_sfw = tmem + 256, t_sfx = tmem + 264;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ TMA producer
+            uint32_t j = 0;
+            for (uint32_t u = u_begin; u < u_end; ++u, ++j) {
+                const uint32_t tile = u / num_kb;
+                const int kb = static_cast<int>(u - tile * num_kb);
+                const int s = j % S;
+                if (j >= static_cast<uint32_t>(S) && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) break;
+                mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
+                tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
+                tma_load_2d(sX(s), &xmap, &full_bar[s], kb * kBKBytes, 0);
+                tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
+                tma_load_5d(sSfx(s), &sfxmap, &full_bar[s], 0, 0, 0, 0, 2 * kb);
+            }
+            for (uint32_t i = (j > static_cast<uint32_t>(S) ? j - S : 0); i < j; ++i)
+                if (!mbar_wait(&full_bar[i % S], (i / S) & 1, kDrainLimitNs)) break;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ MMA issuer
+            const uint32_t idesc_lo = idesc_mxf4(mp, 0), idesc_hi = idesc_mxf4(mp, 2);
+            uint32_t j = 0, piece = 0;
+            bool stop = false;
+            for (uint32_t u = u_begin; u < u_end && !stop; ++piece) {
+                const uint32_t tile = u / num_kb;
+                const uint32_t u_stop = min(u_end, (tile + 1) * num_kb);
+                const int b = piece & 1;
+                if (piece >= 2 && !mbar_wait_or_abort(&accum_empty[b], ((piece >> 1) - 1) & 1, limit, &failed)) break;
+                tc_fence_after();
+                for (bool first = true; u < u_stop; ++u, ++j, first = false) {
+                    const int s = j % S;
+                    if (!mbar_wait_or_abort(&full_bar[s], (j / S) & 1, limit, &failed)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    tc_cp_sf_wide(t_sfw, sdesc_sf_wide(smem_u32(sSfw(s))));
+                    tc_cp_sf_wide(t_sfx, sdesc_sf_wide(smem_u32(sSfx(s))));
+                    const uint64_t wdesc = sdesc_sw128(smem_u32(sW(s)));
+                    const uint64_t xdesc = sdesc_sw128(smem_u32(sX(s)));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c = q >> 1;
+                        tc_mma_mxf4(tmem + 128 * b, wdesc + 2 * q, xdesc + 2 * q, (q & 1) ? idesc_hi : idesc_lo,
+                                    t_sfw + 4 * c, t_sfx + 4 * c, (first && q == 0) ? 0u : 1u);
+                    }
+                    tc_commit(&empty_bar[s]);
+                }
+                tc_commit(&accum_full[b]);
+            }
+            // every MMA issued must be done before TMEM is released
+            tc_commit(&mma_done);
+            mbar_wait(&mma_done, 0, kDrainLimitNs);
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2-5)
+        const int quarter = warp & 3;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int nl = quarter * 32 + lane;          // W row inside the tile
+        uint8_t *ystage = sY + static_cast<size_t>(quarter) * mp * 64;  // [mp][32] bf16 of this warp
+        uint32_t piece = 0;
+        for (uint32_t u = u_begin; u < u_end; ++piece) {
+            const uint32_t tile = u / num_kb;
+            const uint32_t u_first = tile * num_kb;
+            const uint32_t u_stop = min(u_end, u_first + num_kb);
+            const uint32_t c_first = cta_of(u_first), c_last = cta_of(u_first + num_kb - 1);
+            const int npieces = static_cast<int>(c_last - c_first + 1);
+            const int pidx = static_cast<int>(blockIdx.x - c_first);
+            u = u_stop;
+            const int b = piece & 1;
+            if (!mbar_wait_or_abort(&accum_full[b], (piece >> 1) & 1, limit, &failed)) break;
+            tc_fence_after();
+            if (failed) break;
+            const int64_t n = static_cast<int64_t>(tile) * 128 + nl;
+            const bool staged = npieces == 1 && !g.out_f32;
+            if (staged) {  // the previous tile's store (issued by lane 0) has read the staging buffer
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+            }
+            float *part = g.partials + ((static_cast<uint64_t>(tile) * g.max_pieces + pidx) * g.M) * 128;
+            auto emit = [&](int m0, const uint32_t (&v)[32]) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int m = m0 + i;
+                    const float f = __uint_as_float(v[i]);
+                    if (staged) {
+                        if (m < mp) reinterpret_cast<__nv_bfloat16 *>(ystage)[m * 32 + lane] = __float2bfloat16_rn(f);
+                    } else if (m < g.M) {
+                        if (npieces == 1) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = f;
+                        else __stcg(part + static_cast<int64_t>(m) * 128 + nl, f);
+                    }
+                }
+            };
+            for (int m0 = 0; m0 < mp; m0 += 64) {  // two TMEM loads in flight per wait
+                uint32_t v0[32], v1[32];
+                tmem_ld32(taddr + 128 * b + m0, v0);
+                if (m0 + 32 < mp) tmem_ld32(taddr + 128 * b + m0 + 32, v1);
+                tmem_ld_wait();
+                emit(m0, v0);
+                if (m0 + 32 < mp) emit(m0 + 32, v1);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accum_empty[b]);
+            if (staged) {
+                fence_proxy_async_smem();  // generic writes -> the TMA store's reads
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&ymap, ystage, static_cast<int32_t>(tile * 128 + quarter * 32), 0);
+                    bulk_commit();
+                }
+            }
+            if (npieces > 1) {
+                // publish this piece, then let the CTA that completes the tile add the pieces in order.
+                // The barrier orders every thread's partial stores before thread 0's fence and count
+                // increment (a cumulative release); the reader side mirrors it.
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (warp == 2 && lane == 0) {
+                    __threadfence();
+                    s_last = atomicAdd(&g.counts[tile], 1) == npieces - 1;
+                    __threadfence();
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (s_last) {
+                    float *base = g.partials + (static_cast<uint64_t>(tile) * g.max_pieces) * g.M * 128 + nl;
+                    for (int m0 = 0; m0 < g.M; m0 += 16) {
+                        float acc[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+                        for (int p = 0; p < npieces; ++p) {  // 16 independent loads per piece: one round trip
+                            float v[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                v[i] = (m0 + i < g.M) ? __ldcg(base + (static_cast<uint64_t>(p) * g.M + m0 + i) * 128) : 0.0f;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) acc[i] += v[i];
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int m = m0 + i;
+                            if (m >= g.M) break;
+                            if (g.out_f32) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = acc[i];
+                            else static_cast<__nv_bfloat16 *>(g.y)[static_cast<int64_t>(m) * g.N + n] = __float2bfloat16_rn(acc[i]);
+                        }
+                        for (int p = 0; p < npieces; ++p)  // the workspace goes back to all-zero
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (m0 + i < g.M) __stcg(base + (static_cast<uint64_t>(p) * g.M + m0 + i) * 128, 0.0f);
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (warp == 2 && lane == 0) g.counts[tile] = 0;  // ready for the next call
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 }  // namespace macaq

@@ -240,8 +240,104 @@ macaq_status run_gemm(const CUtensorMap &amap, const CUtensorMap &bmap, const Ge
     return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
 }
 
+// ------------------------------------------------------------------------ skinny GEMM (M <= 128)
+constexpr int kSkinnyMaxM = 128;
+
+struct SkinnyPlan {
+    int32_t mp, stages, max_pieces;
+    uint32_t units, gran, ctas, tiles;
+    size_t partial_bytes, count_bytes;
+};
+
+// Work split of the skinny GEMM on a device with `sms` SMs: equal contiguous unit ranges per CTA,
+// cut either anywhere (tiles split over CTAs, partial sums through the workspace) or on tile
+// boundaries (no partials), whichever moves fewer bytes per SM.
+SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms) {
+    SkinnyPlan p{};
+    p.mp = static_cast<int32_t>((M + 15) / 16 * 16);
+    p.tiles = static_cast<uint32_t>(N / 128);
+    const uint32_t num_kb = static_cast<uint32_t>(K / 256);
+    p.units = p.tiles * num_kb;
+    const double w_bytes = static_cast<double>(N) * K * 0.53125;
+    const uint32_t whole_ctas = p.tiles < static_cast<uint32_t>(sms) ? p.tiles : static_cast<uint32_t>(sms);
+    const double whole_cost = w_bytes / whole_ctas * ((p.tiles + whole_ctas - 1) / whole_ctas) / (static_cast<double>(p.tiles) / whole_ctas);
+    const uint32_t split_ctas = p.units < static_cast<uint32_t>(sms) ? p.units : static_cast<uint32_t>(sms);
+    const double pieces = p.tiles + split_ctas;  // every range boundary adds at most one piece
+    // per-SM bytes, plus the partial traffic (write, read, zero) and the serial cross-CTA reduction at
+    // the end (a fence, an atomic and a round trip: about what an SM streams in 2.5 us)
+    const double split_cost = (w_bytes + 3.0 * pieces * M * 128 * 4) / split_ctas + 125.0e3;
+    const bool split = split_cost < whole_cost;
+    p.gran = split ? 1 : num_kb;
+    p.ctas = split ? split_ctas : whole_ctas;
+    const uint32_t chunks = p.units / p.gran;
+    int max_pieces = 1;
+    for (uint32_t t = 0; t < p.tiles && split; ++t) {
+        const uint64_t u0 = static_cast<uint64_t>(t) * num_kb, u1 = u0 + num_kb - 1;
+        const uint64_t c0 = ((u0 / p.gran + 1) * p.ctas - 1) / chunks, c1 = ((u1 / p.gran + 1) * p.ctas - 1) / chunks;
+        const int np = static_cast<int>(c1 - c0 + 1);
+        if (np > max_pieces) max_pieces = np;
+    }
+    p.max_pieces = max_pieces;
+    p.partial_bytes = split ? static_cast<size_t>(p.tiles) * max_pieces * static_cast<size_t>(M) * 128 * 4 : 0;
+    p.count_bytes = (static_cast<size_t>(p.tiles) * 4 + 255) / 256 * 256;
+    const int smem_budget = 232448 - 1024 - 1024 - skinny_stage_bytes_y(p.mp);  // minus slack, static data, Y staging
+    int st = smem_budget / skinny_stage_bytes(p.mp);
+    p.stages = st > kSkinnyMaxStages ? kSkinnyMaxStages : st;
+    return p;
+}
+
+macaq_status run_skinny(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K, const uint8_t *Wq,
+                        const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace, size_t ws_bytes,
+                        int sms, cudaStream_t st) {
+    const SkinnyPlan p = skinny_plan(M, N, K, sms);
+    if (ws_bytes < p.partial_bytes + p.count_bytes) return MACAQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MACAQ_ERR_ALIGNMENT;
+    CUtensorMap wmap, xmap, sfwmap, sfxmap, ymap;
+    macaq_status s = tensor_map_2d(&wmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s == MACAQ_OK)
+        s = tensor_map_2d(&xmap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, kBKBytes, p.mp,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    // replicated scale factors: (128 B, the K-block's two tiles, 8-row group, replica (stride 0), tile)
+    const uint32_t sbox[5] = {128, 2, 4, 4, 1};
+    const uint64_t sstr[4] = {512, 128, 0, 512};
+    if (s == MACAQ_OK) {
+        const uint64_t d[5] = {128, 2, 4, 4, macaq_sf_bytes(N, K) / 512};
+        s = tensor_map(&sfwmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, d, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    if (s == MACAQ_OK) {
+        const uint64_t d[5] = {128, 2, 4, 4, macaq_sf_bytes(M, K) / 512};
+        s = tensor_map(&sfxmap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, d, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    // Y as bf16 [M, N]; each epilogue warp stores a 32-column x Mp-row box
+    if (s == MACAQ_OK)
+        s = tensor_map_2d(&ymap, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 32, p.mp, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (s != MACAQ_OK) return s;
+    SkinnyArgs g;
+    g.y = Y;
+    g.counts = static_cast<int32_t *>(workspace);
+    g.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + p.count_bytes);
+    g.M = static_cast<int32_t>(M);
+    g.N = static_cast<int32_t>(N);
+    g.K = static_cast<int32_t>(K);
+    g.mp = p.mp;
+    g.out_f32 = out_dtype == MACAQ_OUT_F32;
+    g.stages = p.stages;
+    g.max_pieces = p.max_pieces;
+    g.units = p.units;
+    g.gran = p.gran;
+    g.wait_limit_ns = g_wait_limit_ns.load();
+    const size_t smem = 1024 + static_cast<size_t>(p.stages) * skinny_stage_bytes(p.mp) + skinny_stage_bytes_y(p.mp);
+    s = set_smem(gemm_mxf4_skinny_kernel, smem);
+    if (s != MACAQ_OK) return s;
+    gemm_mxf4_skinny_kernel<<<p.ctas, 192, smem, st>>>(wmap, xmap, sfwmap, sfxmap, ymap, g);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+}
+
 macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, int32_t E, int64_t rows, int64_t N,
-                  int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, cudaStream_t st) {
+                  int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
+                  size_t ws_bytes, cudaStream_t st) {
     if (rows < 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 128 != 0) return MACAQ_ERR_SHAPE;
     if (rows >= (int64_t(1) << 31) || static_cast<int64_t>(E) * N >= (int64_t(1) << 31)) return MACAQ_ERR_SHAPE;
     if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
@@ -255,6 +351,9 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
     DeviceInfo dev;
     macaq_status s = device_info(&dev);
     if (s != MACAQ_OK) return s;
+
+    if (offsets == nullptr && rows <= kSkinnyMaxM && K % 256 == 0 && workspace != nullptr)
+        return run_skinny(A, Asf, rows, N, K, Wq, Wsf, Y, out_dtype, workspace, ws_bytes, dev.sms, st);
 
     const int BN = (N % 256 == 0) ? 256 : 128;
     const bool grouped = offsets != nullptr;
@@ -380,8 +479,12 @@ size_t macaq_grouped_sf_bytes(int64_t total_rows, int32_t E, int64_t K) {
 }
 
 size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E) {
-    (void)M, (void)N, (void)K, (void)E;
-    return 0;
+    if (E != 0 || M <= 0 || M > macaq::kSkinnyMaxM || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0) return 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    const macaq::SkinnyPlan p = macaq::skinny_plan(M, N, K, sms);
+    return p.partial_bytes + p.count_bytes;
 }
 
 macaq_status macaq_prep_weights(const void *W, const float *s, int64_t N, int64_t K, int32_t had_block, uint8_t *Wq,
@@ -401,11 +504,11 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
 macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M, int64_t N,
                           int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
                           int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
-    (void)inv_s, (void)had_block, (void)workspace, (void)ws_bytes;
+    (void)inv_s, (void)had_block;
     if (mode == MACAQ_A_BF16_FUSED) return MACAQ_ERR_UNSUPPORTED;
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
-    return macaq::gemm(static_cast<const uint8_t *>(A), Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype,
-                       static_cast<cudaStream_t>(stream));
+    return macaq::gemm(static_cast<const uint8_t *>(A), Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, workspace,
+                       ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
@@ -416,7 +519,7 @@ macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *As
     if (mode != MACAQ_A_QUANTIZED) return mode == MACAQ_A_BF16_FUSED ? MACAQ_ERR_UNSUPPORTED : MACAQ_ERR_INVALID_ARG;
     if (group_offsets == nullptr) return MACAQ_ERR_INVALID_ARG;
     return macaq::gemm(static_cast<const uint8_t *>(A), Asf, group_offsets, E, total_rows, N, K, Wq, Wsf, Y,
-                       out_dtype, static_cast<cudaStream_t>(stream));
+                       out_dtype, nullptr, 0, static_cast<cudaStream_t>(stream));
 }
 
 macaq_status macaq_device_status(int32_t *status_out, int32_t reset) {
