@@ -159,6 +159,34 @@ macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const
                           void *Y, int32_t out_dtype, void *workspace, size_t ws_bytes,
                           macaq_stream_t stream);
 
+/* Size of the library's own fixed scratch area used by macaq_linear_fixed_scratch (8 MiB). */
+#define MACAQ_FIXED_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * macaq_linear without a caller-supplied workspace and without allocating device memory.
+ * The method on the pages has no counterpart of this call: it exists for callers that cannot
+ * allocate device memory at call time, such as a host that has handed all device memory to its
+ * own pool, an embedding in a C program without a device allocator, or a serving loop in which an
+ * allocation would synchronize the device and stall the other streams.
+ * Arguments, results and errors are those of macaq_linear without workspace/ws_bytes. Dense calls
+ * with M <= 128 and K % 256 == 0 run the skinny kernel on a scratch area that lives in the
+ * library's static device data (MACAQ_FIXED_SCRATCH_BYTES per device); every other shape runs the
+ * general kernels, which need no scratch.
+ *   - The first call on each device looks the scratch's address up (with that device current) and
+ *     may load the module; make that first call before any stream capture.
+ *   - Sizes whose skinny plan needs more than MACAQ_FIXED_SCRATCH_BYTES (what
+ *     macaq_workspace_bytes(M, N, K, 0) reports) are rejected with MACAQ_ERR_WORKSPACE before
+ *     anything is launched.
+ *   - Only the per-tile counters must start at zero; each call clears them on `stream` (a memset of
+ *     at most a few KB) before its kernel, so a call after a MACAQ_ERR_TIMEOUT needs no clean-up.
+ *   - All calls on one device share the one scratch area: two calls whose kernels may overlap
+ *     (different streams, or different host threads without ordering) race and give wrong results.
+ *     Order them on one stream, or use macaq_linear with separate workspaces.
+ */
+macaq_status macaq_linear_fixed_scratch(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
+                                        int64_t M, int64_t N, int64_t K, int32_t had_block, const uint8_t *Wq,
+                                        const uint8_t *Wsf, void *Y, int32_t out_dtype, macaq_stream_t stream);
+
 /*
  * Grouped (MoE) W4A4 linear: rows [offsets[e], offsets[e+1]) of A are multiplied by expert e's
  * weights. A must already be quantized by macaq_act_quant in grouped form (mode must be

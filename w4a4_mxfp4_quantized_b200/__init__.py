@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "MacaqError", "OUT_BF16", "OUT_F32", "A_QUANTIZED", "A_BF16_FUSED",
     "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "status_str",
-    "prep_weights", "act_quant", "linear", "grouped_linear", "device_status", "set_wait_limit_ns",
+    "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
+    "set_wait_limit_ns",
     "library_path", "lib",
 ]
 
@@ -50,6 +51,8 @@ _SIGNATURES = {
     "macaq_act_quant": ([_vp, _vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
     "macaq_linear": ([_i32, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp, _sz, _vp],
                      ctypes.c_int),
+    "macaq_linear_fixed_scratch": ([_i32, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp],
+                                   ctypes.c_int),
     "macaq_grouped_linear": ([_i32, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp,
                               _sz, _vp], ctypes.c_int),
     "macaq_device_status": ([ctypes.POINTER(ctypes.c_int32), _i32], ctypes.c_int),
@@ -201,6 +204,20 @@ def linear(A: torch.Tensor, Asf: torch.Tensor | None, Wq: torch.Tensor, Wsf: tor
     _check("macaq_linear", lib().macaq_linear(
         mode, _ptr(A), _ptr(Asf), _ptr(inv_s), M, N, K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype,
         _ptr(workspace), ws_bytes, _stream(dev)))
+    return Y
+
+
+def linear_fixed_scratch(A: torch.Tensor, Asf: torch.Tensor, Wq: torch.Tensor, Wsf: torch.Tensor, *,
+                         out_dtype: int = OUT_BF16, Y=None):
+    """linear() on the library's fixed per-device scratch: the C call allocates no device memory
+    (pass Y to allocate nothing here either). Calls that may overlap on one device race."""
+    N = Wq.shape[0]
+    K = Wq.shape[1] * 2
+    M = A.shape[0]
+    dev = A.device
+    Y = _out(M, N, out_dtype, dev, Y)
+    _check("macaq_linear_fixed_scratch", lib().macaq_linear_fixed_scratch(
+        A_QUANTIZED, _ptr(A), _ptr(Asf), None, M, N, K, 32, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype, _stream(dev)))
     return Y
 
 

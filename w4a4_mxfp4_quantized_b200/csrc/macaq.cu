@@ -447,6 +447,52 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
 }
 
 }  // namespace
+// ------------------------------------------------------------------------ fixed scratch
+// Scratch of the skinny kernel for callers that may not allocate device memory: it is part of the
+// module's static device data, so it exists as soon as the module is loaded on a device.
+constexpr int kMaxDevices = 64;
+__device__ __align__(256) uint8_t g_fixed_scratch[MACAQ_FIXED_SCRATCH_BYTES];
+
+// Device address of g_fixed_scratch on the current device, looked up once per device.
+macaq_status fixed_scratch(void **out) {
+    static std::mutex mu;
+    static std::array<void *, kMaxDevices> addr{};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return MACAQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_fixed_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return MACAQ_OK;
+}
+
+macaq_status linear_fixed_scratch(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K,
+                                  const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype,
+                                  cudaStream_t st) {
+    void *scratch = nullptr;
+    macaq_status s = fixed_scratch(&scratch);
+    if (s != MACAQ_OK) return s;
+    const bool skinny = M >= 1 && M <= kSkinnyMaxM && N > 0 && N % 128 == 0 && K > 0 && K % 256 == 0 &&
+                        N < (int64_t(1) << 31) && K < (int64_t(1) << 31);
+    if (!skinny) return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, nullptr, 0, st);
+    if (A == nullptr || Asf == nullptr || Wq == nullptr || Wsf == nullptr || Y == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+    const SkinnyPlan p = skinny_plan(M, N, K, dev.sms);
+    if (p.partial_bytes + p.count_bytes > MACAQ_FIXED_SCRATCH_BYTES) return MACAQ_ERR_WORKSPACE;
+    const cudaError_t e = cudaMemsetAsync(scratch, 0, p.count_bytes, st);  // the per-tile counters
+    if (e != cudaSuccess) return cuda_fail(e);
+    return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, scratch, MACAQ_FIXED_SCRATCH_BYTES, st);
+}
+
 }  // namespace macaq
 
 // ============================================================================ C ABI
@@ -509,6 +555,16 @@ macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
     return macaq::gemm(static_cast<const uint8_t *>(A), Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, workspace,
                        ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_linear_fixed_scratch(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
+                                        int64_t M, int64_t N, int64_t K, int32_t had_block, const uint8_t *Wq,
+                                        const uint8_t *Wsf, void *Y, int32_t out_dtype, macaq_stream_t stream) {
+    (void)inv_s, (void)had_block;
+    if (mode == MACAQ_A_BF16_FUSED) return MACAQ_ERR_UNSUPPORTED;
+    if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
+    return macaq::linear_fixed_scratch(static_cast<const uint8_t *>(A), Asf, M, N, K, Wq, Wsf, Y, out_dtype,
+                                       static_cast<cudaStream_t>(stream));
 }
 
 macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
