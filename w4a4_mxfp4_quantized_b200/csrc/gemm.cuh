@@ -158,6 +158,67 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem, int warp, int lane,
     }
 }
 
+// Epilogue of the 2-SM kernel: this warp's 32 accumulator rows x 128 columns leave TMEM first (the
+// MMA warp gets the columns back at once), then go to Y through a 4 KB staging buffer as TMA stores
+// of 32 rows x 128 bytes, so every write reaches L2 as whole 128-byte lines. The buffer holds 128-byte
+// rows with the 16-byte chunks of row r at chunk position (k ^ r % 8), the TMA 128-byte swizzle, which
+// keeps the warp's shared-memory writes free of bank conflicts. Rows at or past M are clipped by the
+// tensor map.
+__device__ __forceinline__ void store_chunk_tma(const CUtensorMap *ymap, uint8_t *buf, int lane, const uint32_t *w,
+                                                int32_t col, int32_t row) {
+    if (lane == 0) bulk_wait_read();  // the buffer's previous store has been read out
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<uint4 *>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(ymap, buf, col, row);
+        bulk_commit();
+    }
+}
+
+__device__ __forceinline__ void epilogue_tile_pair(uint32_t tmem, int warp, int lane, int32_t row0, int32_t col0,
+                                                   bool out_f32, const CUtensorMap *ymap, uint8_t *buf,
+                                                   uint32_t accum_empty_addr) {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
+    const int32_t row = row0 + quarter * 32;
+    const int32_t col = col0 + half * 128;
+    if (out_f32) {
+        uint32_t v[128];
+        tmem_ld64(taddr, *reinterpret_cast<uint32_t(*)[64]>(v));
+        tmem_ld64(taddr + 64, *reinterpret_cast<uint32_t(*)[64]>(v + 64));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) store_chunk_tma(ymap, buf, lane, v + 32 * c, col + 32 * c, row);
+    } else {
+        uint32_t packed[64];
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+            uint32_t v[64];
+            tmem_ld64(taddr + cb * 64, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                packed[cb * 32 + k] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) store_chunk_tma(ymap, buf, lane, packed + 32 * c, col + 64 * c, row);
+    }
+}
+
 template <int BN, bool kGrouped>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, GemmArgs g) {
@@ -365,12 +426,13 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
 // per-tile accumulator signals go to both CTAs; every epilogue warp of both CTAs releases the
 // accumulator on the leader's accum_empty barrier.
 struct PairCfg {
-    static constexpr int kStages = 5;
+    static constexpr int kStages = 4;
     static constexpr int kABytes = 128 * kBKBytes;      // this CTA's 128 rows of A
     static constexpr int kBBytes = 128 * kBKBytes;      // this CTA's half of the 256 B rows
     static constexpr int kSfxBytes = 12288;             // replicated SF: A 4 KB, then B 4 KB per chunk
     static constexpr int kStageBytes = kABytes + kBBytes + kSfxBytes;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
+    static constexpr int kEpiBytes = kEpiWarps * 4096;  // one 32 x 128-byte store buffer per epilogue warp
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes;
     static constexpr int kTmemSfa = 256;
     static constexpr int kTmemSfb = 264;
     static constexpr int kTmemCols = 512;
@@ -380,7 +442,7 @@ struct PairCfg {
 __global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                       const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
-                      GemmArgs g, int sf_replica_boxes) {
+                      const __grid_constant__ CUtensorMap ymap, GemmArgs g, int sf_replica_boxes) {
     using C = PairCfg;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t dsmem[];
@@ -395,6 +457,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     uint8_t *sA = smem;
     uint8_t *sB = sA + S * C::kABytes;
     uint8_t *sSfx = sB + S * C::kBBytes;
+    uint8_t *sEpi = sSfx + S * C::kSfxBytes;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -424,6 +487,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         prefetch_tensor_map(&bmap);
         prefetch_tensor_map(&sfamap);
         prefetch_tensor_map(&sfbmap);
+        prefetch_tensor_map(&ymap);
     }
     if (warp == 1) {
         tmem_alloc_pair(&tmem_slot, C::kTmemCols);
@@ -537,10 +601,10 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
             int leader_failed;
             asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(leader_failed) : "r"(leader_failed_addr) : "memory");
             if (failed || leader_failed) break;
-            const int64_t row0 = static_cast<int64_t>(mt) * 256 + rank * 128;
-            const int64_t row_end = row0 + 128 < g.rows ? row0 + 128 : g.rows;
-            epilogue_tile<256>(tmem, warp, lane, row0, row_end, static_cast<int64_t>(nt) * 256, g, empty_addr);
+            epilogue_tile_pair(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128), static_cast<int32_t>(nt * 256),
+                               g.out_f32 != 0, &ymap, sEpi + (warp - 2) * 4096, empty_addr);
         }
+        if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it
     }
 
     tc_fence_before();

@@ -405,6 +405,13 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
                     s = tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, db4, sb4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
             }
         }
+        // Y in 32-row x 128-byte boxes, 128-byte swizzled (the epilogue's staging layout)
+        CUtensorMap ymap;
+        if (s == MACAQ_OK) {
+            const bool f32 = out_dtype == MACAQ_OUT_F32;
+            s = tensor_map_2d(&ymap, Y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, rows,
+                              N * (f32 ? 4 : 2), f32 ? 32 : 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+        }
         if (s != MACAQ_OK) return s;
         const int64_t tiles = ((rows + 255) / 256) * (N / 256);
         const int64_t max_pairs = dev.sms / 2;
@@ -423,7 +430,7 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_mxf4_pair_kernel, amap, bmap, sfamap, sfbmap, g, replica_boxes);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_mxf4_pair_kernel, amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes);
         if (e != cudaSuccess) return cuda_fail(e);
         e = cudaGetLastError();
         return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
