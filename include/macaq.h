@@ -95,14 +95,22 @@ size_t macaq_grouped_sf_bytes(int64_t total_rows, int32_t E, int64_t K);
 
 /* Workspace bytes macaq_linear can use for these sizes on the current device (E = 0 for dense).
  * Dense calls with M <= 128 and K % 256 == 0 given a workspace of at least this size run the skinny
- * kernel (weights in
- * the MMA's 128-row slot, the unit space split evenly over all SMs, split tiles reduced through the
- * workspace); without a workspace they run the general kernel. 0 means no workspace is used.
- * Contract: the workspace must be all zero before its first use; every call leaves it zero again
- * (per-tile counters reset themselves), so one buffer can serve any number of consecutive calls.
- * Calls that may run at the same time on different streams need separate workspaces. After a call
- * that reported MACAQ_ERR_TIMEOUT, zero the workspace again. */
+ * kernel (weights in the MMA's 128-row slot, the unit space split evenly over all SMs, split tiles
+ * reduced through the workspace); without a workspace they run the general kernel. 0 means no
+ * workspace is used.
+ * Layout and contract: the first MACAQ_WORKSPACE_COUNTER_BYTES hold per-tile arrival counters. They
+ * must be zero before the workspace's first use, and every call leaves them zero again (each counter
+ * is reset by the CTA that consumed it), so one buffer serves any number of consecutive calls of any
+ * shapes. The bytes after them are scratch: no initial value is needed and calls leave arbitrary
+ * data there. Calls that may run at the same time on different streams need separate workspaces.
+ * After a call that reported MACAQ_ERR_TIMEOUT, zero the counter region again. */
+#define MACAQ_WORKSPACE_COUNTER_BYTES ((size_t)65536)
 size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E);
+
+/* Workspace bytes of the fused mode (MACAQ_A_BF16_FUSED) of macaq_linear (E = 0) and
+ * macaq_grouped_linear (E experts): the region above, then room for the quantized activations and
+ * their scale factors where the call quantizes X in a separate pass. Same layout and contract. */
+size_t macaq_fused_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E);
 
 /*
  * Offline weight preparation (the absorbed inverse transform).
@@ -144,9 +152,14 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
  * tensor cores (kind::mxf4 block-scaled MMA), written as bf16 (round-to-nearest-even) or fp32.
  *   mode == MACAQ_A_QUANTIZED:  A = Xq device u8 [M, K/2], Asf = Xsf (tiled, macaq_sf_bytes(M, K)),
  *                               inv_s and had_block are ignored.
- *   mode == MACAQ_A_BF16_FUSED: A = X device bf16 [M, K], inv_s device fp32 [K] (NULL = 1), and the
- *                               kernel applies scale, Hadamard and MXFP4 itself, bit-identical to
- *                               macaq_act_quant; Asf is ignored.
+ *   mode == MACAQ_A_BF16_FUSED: A = X device bf16 [M, K], inv_s device fp32 [K] (NULL = 1), had_block
+ *                               b in {1, 16, 32, 64, 128}; Asf is ignored. The call quantizes X
+ *                               bit-identically to macaq_act_quant, so Y equals macaq_act_quant
+ *                               followed by the quantized mode. M <= 16 with K % 256 == 0: inside the
+ *                               skinny kernel (quantizer warps write the MMA's operand stages; no
+ *                               quantized activation in HBM). Otherwise: a quantizer pass into the
+ *                               workspace, then the GEMM, in stream order. Needs a workspace of
+ *                               macaq_fused_workspace_bytes(M, N, K, 0) bytes (else MACAQ_ERR_WORKSPACE).
  *   Wq, Wsf    from macaq_prep_weights: u8 [N, K/2] and the tiled SF of N rows
  *   Y          device [M, N], bf16 or fp32 per out_dtype (written)
  *   workspace  NULL, or device scratch of at least macaq_workspace_bytes(M, N, K, 0) bytes under the
@@ -189,13 +202,17 @@ macaq_status macaq_linear_fixed_scratch(int32_t mode, const void *A, const uint8
 
 /*
  * Grouped (MoE) W4A4 linear: rows [offsets[e], offsets[e+1]) of A are multiplied by expert e's
- * weights. A must already be quantized by macaq_act_quant in grouped form (mode must be
- * MACAQ_A_QUANTIZED in this version; other modes return MACAQ_ERR_UNSUPPORTED).
- *   A, Asf         Xq [total_rows, K/2] and the grouped tiled SF
+ * weights.
+ *   mode == MACAQ_A_QUANTIZED:  A, Asf = Xq [total_rows, K/2] and the grouped tiled SF from
+ *                               macaq_act_quant in grouped form; inv_s and had_block are ignored.
+ *   mode == MACAQ_A_BF16_FUSED: A = X device bf16 [total_rows, K], inv_s device fp32 [E, K] (NULL = 1),
+ *                               had_block b; the call runs the grouped quantizer into the workspace
+ *                               (macaq_fused_workspace_bytes(total_rows, N, K, E) bytes), then the
+ *                               grouped GEMM. Asf is ignored.
  *   group_offsets  device int32 [E + 1] (as for macaq_act_quant); 1 <= E <= 1024
  *   Wq             device u8 [E, N, K/2];  Wsf device u8 [E, macaq_sf_bytes(N, K)]
  *   Y              device [total_rows, N] (written; only rows of some expert are written)
- *   workspace      unused in this version (may be NULL)
+ *   workspace      quantized mode: unused (may be NULL); fused mode: as above
  * Source: glonce.com page, paragraph 5 (W4A4 grouped matmul).
  */
 macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,

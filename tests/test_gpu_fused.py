@@ -1,0 +1,125 @@
+"""GPU parity of the fused layer (mode A_BF16_FUSED: bf16 X in, the call quantizes it).
+
+The quantization is bit-exact and the GEMM plan is the same as for the quantized mode, so the fused
+result must equal act_quant followed by the quantized linear bit for bit; it is also checked against
+the oracle's pipeline (oracle act_quant, float64 GEMM) within 1e-5 of sum|terms| per element. M <= 16
+with K % 256 == 0 runs the quantizer inside the skinny GEMM kernel; larger M runs the two-pass form.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w4a4_mxfp4_quantized_b200 as mq
+from w4a4_mxfp4_quantized_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+
+
+def layer(seed, M, N, K, b, with_s):
+    c = inputs.dense_case(seed, M, K, N, n_outliers=3, outlier_factor=30.0, w_std=0.02)
+    s = c.s if with_s else None
+    Wq, Wsf, inv = mq.prep_weights(c.W.cuda(), None if s is None else s.cuda(), b)
+    return c, Wq, Wsf, inv
+
+
+def unfused(X, inv, b, Wq, Wsf, out_dtype):
+    Xq, Xsf = mq.act_quant(X, inv, b)
+    return mq.linear(Xq, Xsf, Wq, Wsf, out_dtype=out_dtype)
+
+
+def fused(X, inv, b, Wq, Wsf, out_dtype):
+    return mq.linear(X, None, Wq, Wsf, mode=mq.A_BF16_FUSED, inv_s=inv, had_block=b, out_dtype=out_dtype)
+
+
+def check_against_oracle(c, b, with_s, Wq_gpu, Wsf_gpu, y32, rows=None):
+    """The oracle quantizes X itself; W' comes from the oracle's own weight prep."""
+    s = c.s if with_s else None
+    inv_s = None if s is None else (np.float32(1.0) / s.numpy()).astype(np.float32)
+    Xq, Xsf = oracle.act_quant(c.X, inv_s, b)
+    Wq, Wsf, _ = oracle.prep_weights(c.W, s, b)
+    Y, T = oracle.linear(Xq, Xsf, Wq, Wsf, rows=rows)
+    y = y32.double().cpu().numpy()
+    if rows is not None:
+        y = y[rows]
+    err = np.abs(y - Y)
+    assert np.all(err <= RTOL * T + 1e-30), f"worst rel {np.max(err / (T + 1e-30)):.3g}"
+
+
+@pytest.mark.parametrize("b", [1, 16, 32, 64, 128])
+@pytest.mark.parametrize("with_s", [True, False])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (5, 512, 1024), (16, 1024, 4096)])
+def test_in_kernel_fusion_equals_two_pass(M, N, K, b, with_s):
+    c, Wq, Wsf, inv = layer(4000 + M + N + K + b, M, N, K, b, with_s)
+    X = c.X.cuda()
+    for out in (mq.OUT_F32, mq.OUT_BF16):
+        ref = unfused(X, inv, b, Wq, Wsf, out)
+        for _ in range(2):  # twice on one workspace: the counters must reset themselves
+            got = fused(X, inv, b, Wq, Wsf, out)
+            torch.cuda.synchronize()
+            assert mq.device_status() == 0
+            assert torch.equal(got.view(torch.int16 if out == mq.OUT_BF16 else torch.int32),
+                               ref.view(torch.int16 if out == mq.OUT_BF16 else torch.int32))
+    check_against_oracle(c, b, with_s, Wq, Wsf, got if out == mq.OUT_F32 else fused(X, inv, b, Wq, Wsf, mq.OUT_F32))
+
+
+@pytest.mark.parametrize("M,N,K", [(17, 512, 1024), (128, 256, 512), (300, 512, 1280), (7, 384, 384)])
+def test_two_pass_fusion(M, N, K):
+    """Shapes outside the in-kernel form (M > 16, or K % 256 != 0): quantizer pass + GEMM."""
+    b = 32
+    c, Wq, Wsf, inv = layer(5000 + M + N + K, M, N, K, b, True)
+    X = c.X.cuda()
+    ref = unfused(X, inv, b, Wq, Wsf, mq.OUT_F32)
+    got = fused(X, inv, b, Wq, Wsf, mq.OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int32), ref.view(torch.int32))
+    check_against_oracle(c, b, True, Wq, Wsf, got)
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_llama3_8b_up_decode_fused(M):
+    c = inputs.llama3_8b_up(M)
+    Wq, Wsf, inv = mq.prep_weights(c.W.cuda(), c.s.cuda(), 32)
+    X = c.X.cuda()
+    ref = unfused(X, inv, 32, Wq, Wsf, mq.OUT_BF16)
+    got = fused(X, inv, 32, Wq, Wsf, mq.OUT_BF16)
+    y32 = fused(X, inv, 32, Wq, Wsf, mq.OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), got.view(torch.int16))
+    check_against_oracle(c, 32, True, Wq, Wsf, y32, rows=np.unique([0, M - 1]))
+
+
+def test_grouped_fused_equals_two_pass():
+    m = inputs.moe_30b_a3b(64, "gate_up")
+    E = m.offsets.numel() - 1
+    K = m.X.shape[1]
+    W = m.W.cuda()
+    N = W.shape[1]
+    Wq = torch.empty(E, N, K // 2, dtype=torch.uint8, device="cuda")
+    Wsf = torch.empty(E, mq.sf_bytes(N, K), dtype=torch.uint8, device="cuda")
+    inv = torch.empty(E, K, dtype=torch.float32, device="cuda")
+    for e in range(E):
+        mq.prep_weights(W[e], m.s[e].cuda(), 32, Wq=Wq[e], Wsf=Wsf[e], inv_s=inv[e])
+    X, off = m.X.cuda(), m.offsets.cuda()
+    Xq, Xsf = mq.act_quant(X, inv, 32, group_offsets=off)
+    ref = mq.grouped_linear(Xq, Xsf, off, Wq, Wsf, out_dtype=mq.OUT_F32)
+    got = mq.grouped_linear(X, None, off, Wq, Wsf, mode=mq.A_BF16_FUSED, inv_s=inv, had_block=32,
+                            out_dtype=mq.OUT_F32)
+    torch.cuda.synchronize()
+    rows = np.arange(int(m.offsets[-1]))
+    assert torch.equal(got[rows].view(torch.int32), ref[rows].view(torch.int32))
+
+
+def test_fused_needs_a_workspace():
+    c, Wq, Wsf, inv = layer(77, 4, 256, 256, 32, True)
+    X = c.X.cuda()
+    Y = torch.empty(4, 256, dtype=torch.bfloat16, device="cuda")
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    status = mq.lib().macaq_linear(mq.A_BF16_FUSED, X.data_ptr(), None, inv.data_ptr(), 4, 256, 256, 32,
+                                   Wq.data_ptr(), Wsf.data_ptr(), Y.data_ptr(), mq.OUT_BF16, None, 0, st)
+    assert mq.status_str(status) == "MACAQ_ERR_WORKSPACE"
+    assert mq.fused_workspace_bytes(4, 256, 256) > mq.WORKSPACE_COUNTER_BYTES

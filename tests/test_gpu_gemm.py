@@ -84,16 +84,16 @@ def test_skinny_split_tiles(M, N, K):
     for _ in range(3):
         check_dense(*ops)
     ws = mq._workspace(torch.device("cuda"), 0)
-    assert int(ws.count_nonzero()) == 0
+    assert int(ws[:mq.WORKSPACE_COUNTER_BYTES].count_nonzero()) == 0
 
 
 def test_skinny_shared_workspace_across_shapes():
-    """Calls of different shapes share one workspace, whose layout (counts, then partials) moves with
-    N: each call must leave it all-zero so that the next call's counters start at zero."""
+    """Calls of different shapes share one workspace: each call must leave the counter region zero so
+    that the next call's counters start at zero, whatever it left in the scratch behind them."""
     for M, N, K in [(1, 7168, 4096), (1, 14336, 2048), (3, 256, 4096), (1, 14336, 4096), (16, 1024, 5120)]:
         check_dense(*random_operands(M + N + K, M, N, K), rows=np.array([0, M - 1]))
         ws = mq._workspace(torch.device("cuda"), 0)
-        assert int(ws.count_nonzero()) == 0, (M, N, K)
+        assert int(ws[:mq.WORKSPACE_COUNTER_BYTES].count_nonzero()) == 0, (M, N, K)
 
 
 def test_extreme_scales_and_codes():

@@ -22,7 +22,8 @@ import torch
 
 __all__ = [
     "MacaqError", "OUT_BF16", "OUT_F32", "A_QUANTIZED", "A_BF16_FUSED",
-    "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "status_str",
+    "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "fused_workspace_bytes", "WORKSPACE_COUNTER_BYTES",
+    "status_str",
     "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
     "set_wait_limit_ns",
     "library_path", "lib",
@@ -34,6 +35,7 @@ _lock = threading.Lock()
 _lib = None
 
 OUT_BF16, OUT_F32 = 0, 1
+WORKSPACE_COUNTER_BYTES = 65536  # MACAQ_WORKSPACE_COUNTER_BYTES: the zero-between-calls counter region
 A_QUANTIZED, A_BF16_FUSED = 0, 1
 
 _vp = ctypes.c_void_p
@@ -47,6 +49,7 @@ _SIGNATURES = {
     "macaq_sf_bytes": ([_i64, _i64], _sz),
     "macaq_grouped_sf_bytes": ([_i64, _i32, _i64], _sz),
     "macaq_workspace_bytes": ([_i64, _i64, _i64, _i32], _sz),
+    "macaq_fused_workspace_bytes": ([_i64, _i64, _i64, _i32], _sz),
     "macaq_prep_weights": ([_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
     "macaq_act_quant": ([_vp, _vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
     "macaq_linear": ([_i32, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp, _sz, _vp],
@@ -122,8 +125,9 @@ _ws_cache: dict = {}
 
 
 def _workspace(dev, nbytes: int) -> torch.Tensor:
-    """A zero-initialised scratch buffer per device, grown on demand and reused across calls (the
-    kernels leave it zeroed). Calls that may overlap on different streams need their own buffers."""
+    """A scratch buffer per device, zero-initialised, grown on demand and reused across calls (the
+    kernels leave its counter region zero). Calls that may overlap on different streams need their
+    own buffers."""
     key = torch.device(dev).index
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
@@ -143,6 +147,10 @@ def grouped_sf_bytes(total_rows: int, E: int, K: int) -> int:
 
 def workspace_bytes(M: int, N: int, K: int, E: int = 0) -> int:
     return int(lib().macaq_workspace_bytes(M, N, K, E))
+
+
+def fused_workspace_bytes(M: int, N: int, K: int, E: int = 0) -> int:
+    return int(lib().macaq_fused_workspace_bytes(M, N, K, E))
 
 
 def prep_weights(W: torch.Tensor, s: torch.Tensor | None, had_block: int = 32, *, Wq=None, Wsf=None,
@@ -190,20 +198,27 @@ def linear(A: torch.Tensor, Asf: torch.Tensor | None, Wq: torch.Tensor, Wsf: tor
            out_dtype: int = OUT_BF16, Y=None, workspace=None, use_workspace: bool = True):
     """Dense W4A4 linear Y = dq(A) dq(W')^T (fp32 accumulate; bf16 or fp32 out).
 
-    With few rows (M <= 128) a workspace selects the skinny kernel (weights in the MMA's M slot,
-    split over all SMs); use_workspace=False runs the general kernel instead."""
+    mode=A_QUANTIZED: A, Asf from act_quant. With few rows (M <= 128) a workspace selects the skinny
+    kernel (weights in the MMA's M slot, split over all SMs); use_workspace=False runs the general
+    kernel instead.
+    mode=A_BF16_FUSED: A is bf16 X [M, K]; the call applies inv_s, H_b and MXFP4 itself (inside the
+    GEMM kernel for M <= 16) and needs a workspace."""
     N = Wq.shape[0]
     K = Wq.shape[1] * 2
     M = A.shape[0]
     dev = A.device
     Y = _out(M, N, out_dtype, dev, Y)
-    ws_need = workspace_bytes(M, N, K, 0) if use_workspace else 0
+    fused = mode == A_BF16_FUSED
+    if fused:
+        ws_need = fused_workspace_bytes(M, N, K, 0)
+    else:
+        ws_need = workspace_bytes(M, N, K, 0) if use_workspace else 0
     if workspace is None and ws_need > 0:
         workspace = _workspace(dev, ws_need)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("macaq_linear", lib().macaq_linear(
-        mode, _ptr(A), _ptr(Asf), _ptr(inv_s), M, N, K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype,
-        _ptr(workspace), ws_bytes, _stream(dev)))
+        mode, _ptr(A), None if fused else _ptr(Asf), _ptr(inv_s) if fused else None, M, N, K, had_block, _ptr(Wq),
+        _ptr(Wsf), _ptr(Y), out_dtype, _ptr(workspace), ws_bytes, _stream(dev)))
     return Y
 
 
@@ -221,21 +236,26 @@ def linear_fixed_scratch(A: torch.Tensor, Asf: torch.Tensor, Wq: torch.Tensor, W
     return Y
 
 
-def grouped_linear(A: torch.Tensor, Asf: torch.Tensor, group_offsets: torch.Tensor, Wq: torch.Tensor,
-                   Wsf: torch.Tensor, *, out_dtype: int = OUT_BF16, Y=None, workspace=None):
-    """Grouped W4A4 linear: rows of expert e times W'_e. Wq [E, N, K/2], Wsf [E, sf_bytes(N, K)]."""
+def grouped_linear(A: torch.Tensor, Asf: torch.Tensor | None, group_offsets: torch.Tensor, Wq: torch.Tensor,
+                   Wsf: torch.Tensor, *, mode: int = A_QUANTIZED, inv_s: torch.Tensor | None = None,
+                   had_block: int = 32, out_dtype: int = OUT_BF16, Y=None, workspace=None):
+    """Grouped W4A4 linear: rows of expert e times W'_e. Wq [E, N, K/2], Wsf [E, sf_bytes(N, K)].
+
+    mode=A_BF16_FUSED: A is bf16 X [total_rows, K] and inv_s [E, K]; the call quantizes it per
+    expert into the workspace, then runs the grouped GEMM."""
     E, N, K2 = Wq.shape
     K = K2 * 2
     M = A.shape[0]
     dev = A.device
     Y = _out(M, N, out_dtype, dev, Y)
-    ws_need = workspace_bytes(M, N, K, E)
+    fused = mode == A_BF16_FUSED
+    ws_need = fused_workspace_bytes(M, N, K, E) if fused else workspace_bytes(M, N, K, E)
     if workspace is None and ws_need > 0:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+        workspace = _workspace(dev, ws_need)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("macaq_grouped_linear", lib().macaq_grouped_linear(
-        A_QUANTIZED, _ptr(A), _ptr(Asf), None, _ptr(group_offsets), E, M, N, K, 32, _ptr(Wq), _ptr(Wsf), _ptr(Y),
-        out_dtype, _ptr(workspace), ws_bytes, _stream(dev)))
+        mode, _ptr(A), None if fused else _ptr(Asf), _ptr(inv_s) if fused else None, _ptr(group_offsets), E, M, N,
+        K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype, _ptr(workspace), ws_bytes, _stream(dev)))
     return Y
 
 

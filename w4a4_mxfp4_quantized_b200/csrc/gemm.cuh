@@ -30,6 +30,7 @@
 
 #include "groups.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace macaq {
 
@@ -622,18 +623,29 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
 // of bytes. A CTA's range covers pieces of one or more tiles; a tile covered by one CTA is written
 // straight to Y (bf16 through shared memory and a TMA store), otherwise each piece's fp32 partial goes
 // to the workspace and the CTA that completes the tile's last piece (an atomic count per tile) adds
-// the pieces in their fixed order, writes Y and sets the partials and the count back to zero, so the
-// workspace is all-zero between calls whatever the shapes of earlier calls. When splitting tiles
+// the pieces in their fixed order, writes Y and sets the count back to zero. The counters live in the
+// workspace's first 64 KiB, which is therefore zero between calls whatever the shapes of earlier
+// calls; the partials behind them are written before they are read. When splitting tiles
 // would move more partial bytes than it saves (large M), the ranges are cut on whole tiles instead.
 // Both operands' scale factors arrive replicated (zero-stride TMA view) and go to TMEM with one wide
 // 128x256b copy each per K-block. The stage ring is as deep as shared memory allows; the accumulator
 // is double-buffered in TMEM. Needs K % 256 == 0.
+//
+// Fused form (kFusedB = Hadamard block b > 0, M <= 16): the activations arrive as bf16 X. Per stage
+// the producer also loads X's K-block (16 rows x 256 bf16 by TMA, zero-filled past M) and the
+// K-block's 256 multipliers 1/s (bulk copy); four quantizer warps (warps 6-9, one 32-element group
+// per thread: row t / 8, group t % 8) apply scale, Hadamard and MXFP4 exactly as the quantizer kernel
+// does, and write the codes (128-byte swizzled, as the MMA's descriptor reads them) and the E8M0
+// exponents (four-fold replicated, as the wide copy reads them) straight into the stage. No quantized
+// activation ever goes to HBM. Source: the aipolix.com page, paragraph 2 (transform on each layer's
+// activations at inference); glonce.com page, paragraph 5 (W4A4 dense matmul).
 constexpr int kSkinnyMaxStages = 12;
+constexpr int kSkinnyFusedMaxM = 16;
 
 struct SkinnyArgs {
     void *y;                   // [M, N]
-    float *partials;           // [tiles][max_pieces][M][128] fp32
-    int32_t *counts;           // [tiles], zero between calls
+    float *partials;           // [tiles][max_pieces][M][128] fp32, written before read
+    int32_t *counts;           // [tiles], zero between calls (the workspace's first 64 KiB)
     int32_t M, N, K;
     int32_t mp;                // M rounded up to 16: the MMA's N
     int32_t out_f32;
@@ -642,18 +654,23 @@ struct SkinnyArgs {
     uint32_t units;            // (N / 128) * (K / 256)
     uint32_t gran;             // units per indivisible chunk: 1 (split tiles) or K-blocks per tile (whole tiles)
     uint64_t wait_limit_ns;
+    const float *inv_s;        // fused form: [K] multipliers 1/s, or nullptr for s = 1
 };
 
 __host__ __device__ constexpr int skinny_stage_bytes(int mp) { return 128 * kBKBytes + mp * kBKBytes + 8192; }
+// fused form: + the K-block of bf16 X (mp rows x 512 bytes) and of the multipliers (1 KB)
+__host__ __device__ constexpr int skinny_stage_bytes_fused(int mp) { return skinny_stage_bytes(mp) + mp * 512 + 1024; }
 __host__ __device__ constexpr int skinny_stage_bytes_y(int mp) { return mp * 128 * 2; }  // bf16 staging of one tile
 
-__global__ void __launch_bounds__(192, 1)
+template <int kFusedB>
+__global__ void __launch_bounds__(kFusedB > 0 ? 320 : 192, 1)
 gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                         const __grid_constant__ CUtensorMap sfwmap, const __grid_constant__ CUtensorMap sfxmap,
                         const __grid_constant__ CUtensorMap ymap, SkinnyArgs g) {
     extern __shared__ uint8_t dsmem[];
     __shared__ uint64_t full_bar[kSkinnyMaxStages];
     __shared__ uint64_t empty_bar[kSkinnyMaxStages];
+    __shared__ uint64_t xin_bar[kSkinnyMaxStages];   // fused form: X and 1/s of the stage have landed
     __shared__ uint64_t accum_full[2];
     __shared__ uint64_t accum_empty[2];
     __shared__ uint64_t mma_done;
@@ -661,15 +678,18 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
     __shared__ int32_t s_last;
     __shared__ volatile int failed;
 
+    constexpr bool kFused = kFusedB > 0;
     const int S = g.stages;
     const int mp = g.mp;
-    const int stage_bytes = skinny_stage_bytes(mp);
+    const int stage_bytes = kFused ? skinny_stage_bytes_fused(mp) : skinny_stage_bytes(mp);
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint8_t *sY = smem + S * stage_bytes;  // [4 warps][mp rows][32 columns] bf16
     auto sW = [&](int s) { return smem + s * stage_bytes; };
     auto sX = [&](int s) { return smem + s * stage_bytes + 128 * kBKBytes; };
     auto sSfw = [&](int s) { return smem + s * stage_bytes + (128 + mp) * kBKBytes; };
     auto sSfx = [&](int s) { return smem + s * stage_bytes + (128 + mp) * kBKBytes + 4096; };
+    auto sXin = [&](int s) { return smem + s * stage_bytes + skinny_stage_bytes(mp); };
+    auto sInv = [&](int s) { return smem + s * stage_bytes + skinny_stage_bytes(mp) + mp * 512; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -688,8 +708,9 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], kFused ? 5 : 1);   // fused: the producer and the four quantizer warps
             mbar_init(&empty_bar[s], 1);
+            mbar_init(&xin_bar[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accum_full[b], 1);
@@ -707,6 +728,14 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
         tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
+    if constexpr (kFused) {
+        // the quantizer writes only the scale bytes of rows < 16; the rest of each replicated block
+        // stays zero for the whole launch
+        for (int s = 0; s < S; ++s)
+            for (int i = threadIdx.x; i < 4096 / 16; i += blockDim.x)
+                reinterpret_cast<uint4 *>(sSfx(s))[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -722,11 +751,21 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
                 const int kb = static_cast<int>(u - tile * num_kb);
                 const int s = j % S;
                 if (j >= static_cast<uint32_t>(S) && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) break;
-                mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
-                tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
-                tma_load_2d(sX(s), &xmap, &full_bar[s], kb * kBKBytes, 0);
-                tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
-                tma_load_5d(sSfx(s), &sfxmap, &full_bar[s], 0, 0, 0, 0, 2 * kb);
+                if constexpr (kFused) {
+                    mbar_arrive_expect_tx(&full_bar[s], 128 * kBKBytes + 4096);
+                    tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
+                    tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
+                    // X's K-block as bf16 (rows past M read as zero) and its 256 multipliers
+                    mbar_arrive_expect_tx(&xin_bar[s], mp * 512 + (g.inv_s != nullptr ? 1024 : 0));
+                    tma_load_2d(sXin(s), &xmap, &xin_bar[s], kb * 256, 0);
+                    if (g.inv_s != nullptr) bulk_load(sInv(s), g.inv_s + kb * 256, 1024, &xin_bar[s]);
+                } else {
+                    mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
+                    tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
+                    tma_load_2d(sX(s), &xmap, &full_bar[s], kb * kBKBytes, 0);
+                    tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
+                    tma_load_5d(sSfx(s), &sfxmap, &full_bar[s], 0, 0, 0, 0, 2 * kb);
+                }
             }
             for (uint32_t i = (j > static_cast<uint32_t>(S) ? j - S : 0); i < j; ++i)
                 if (!mbar_wait(&full_bar[i % S], (i / S) & 1, kDrainLimitNs)) break;
@@ -767,6 +806,47 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
             // every MMA issued must be done before TMEM is released
             tc_commit(&mma_done);
             mbar_wait(&mma_done, 0, kDrainLimitNs);
+        }
+    } else if (kFused && warp >= 6) {
+        // ---------------------------------------------------------------- quantizer (fused form)
+        const int t = threadIdx.x - 192;      // 0..127
+        const int m = t >> 3;                 // activation row (< 16)
+        const int gq = t & 7;                 // 32-element group inside the K-block
+        uint32_t j = 0;
+        for (uint32_t u = u_begin; u < u_end; ++u, ++j) {
+            const int s = j % S;
+            // the whole warp leaves together if any lane's wait ran out (the Hadamard may shuffle)
+            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&xin_bar[s], (j / S) & 1, limit, &failed))) break;
+            const uint8_t *src = sXin(s) + m * 512 + gq * 64;
+            uint4 raw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) raw[i] = *reinterpret_cast<const uint4 *>(src + i * 16);
+            uint64_t p[16];
+            unpack_bf16x32(raw, p);
+            if (g.inv_s != nullptr) {
+                const float4 *mv4 = reinterpret_cast<const float4 *>(sInv(s) + gq * 128);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 f = mv4[i];
+                    p[2 * i] = mul2(p[2 * i], pk2(f.x, f.y));
+                    p[2 * i + 1] = mul2(p[2 * i + 1], pk2(f.z, f.w));
+                }
+            }
+            uint4 packed;
+            uint32_t E8;
+            transform_quantize_group<kFusedB, false>(p, packed, E8);
+            // codes: row m's 16-byte chunk gq of the 128-byte row, 128-byte swizzle
+            *reinterpret_cast<uint4 *>(sX(s) + m * 128 + ((gq ^ (m & 7)) << 4)) = packed;
+            // exponent: SF tile half gq / 4, column gq % 4, row m (lane m of 32, row quarter 0), in each
+            // of the four replicas (1 KB apart)
+            uint8_t *sf = sSfx(s) + ((m >> 3) * 2 + (gq >> 2)) * 128 + (m & 7) * 16 + (gq & 3);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sf[q * 1024] = static_cast<uint8_t>(E8);
+            // the stage's input has been read and its operands written: order both before the MMA's
+            // (async-proxy) reads and the next TMA write of the stage
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_bar[s]);
         }
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2-5)
@@ -858,10 +938,6 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
                             if (g.out_f32) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = acc[i];
                             else static_cast<__nv_bfloat16 *>(g.y)[static_cast<int64_t>(m) * g.N + n] = __float2bfloat16_rn(acc[i]);
                         }
-                        for (int p = 0; p < npieces; ++p)  // the workspace goes back to all-zero
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (m0 + i < g.M) __stcg(base + (static_cast<uint64_t>(p) * g.M + m0 + i) * 128, 0.0f);
                     }
                     asm volatile("bar.sync 1, 128;" ::: "memory");
                     if (warp == 2 && lane == 0) g.counts[tile] = 0;  // ready for the next call

@@ -242,8 +242,13 @@ macaq_status run_gemm(const CUtensorMap &amap, const CUtensorMap &bmap, const Ge
 
 // ------------------------------------------------------------------------ skinny GEMM (M <= 128)
 constexpr int kSkinnyMaxM = 128;
+// Workspace layout: per-tile arrival counters in the first 64 KiB (zero between calls; the kernel
+// resets every counter it used), then scratch that needs no initial value: the skinny kernel's fp32
+// partial tiles, and in the fused two-kernel path the quantized activations after them.
+constexpr size_t kCountRegion = 65536;
 
 struct SkinnyPlan {
+    bool ok;                   // the tiles' counters fit the counter region
     int32_t mp, stages, max_pieces;
     uint32_t units, gran, ctas, tiles;
     size_t partial_bytes, count_bytes;
@@ -252,7 +257,7 @@ struct SkinnyPlan {
 // Work split of the skinny GEMM on a device with `sms` SMs: equal contiguous unit ranges per CTA,
 // cut either anywhere (tiles split over CTAs, partial sums through the workspace) or on tile
 // boundaries (no partials), whichever moves fewer bytes per SM.
-SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms) {
+SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms, bool fused = false) {
     SkinnyPlan p{};
     p.mp = static_cast<int32_t>((M + 15) / 16 * 16);
     p.tiles = static_cast<uint32_t>(N / 128);
@@ -263,9 +268,9 @@ SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms) {
     const double whole_cost = w_bytes / whole_ctas * ((p.tiles + whole_ctas - 1) / whole_ctas) / (static_cast<double>(p.tiles) / whole_ctas);
     const uint32_t split_ctas = p.units < static_cast<uint32_t>(sms) ? p.units : static_cast<uint32_t>(sms);
     const double pieces = p.tiles + split_ctas;  // every range boundary adds at most one piece
-    // per-SM bytes, plus the partial traffic (write, read, zero) and the serial cross-CTA reduction at
-    // the end (a fence, an atomic and a round trip: about what an SM streams in 2.5 us)
-    const double split_cost = (w_bytes + 3.0 * pieces * M * 128 * 4) / split_ctas + 125.0e3;
+    // per-SM bytes, plus the partial traffic (write, read) and the serial cross-CTA reduction at the
+    // end (a fence, an atomic and a round trip: about what an SM streams in 2.5 us)
+    const double split_cost = (w_bytes + 2.0 * pieces * M * 128 * 4) / split_ctas + 125.0e3;
     const bool split = split_cost < whole_cost;
     p.gran = split ? 1 : num_kb;
     p.ctas = split ? split_ctas : whole_ctas;
@@ -279,25 +284,48 @@ SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms) {
     }
     p.max_pieces = max_pieces;
     p.partial_bytes = split ? static_cast<size_t>(p.tiles) * max_pieces * static_cast<size_t>(M) * 128 * 4 : 0;
-    p.count_bytes = (static_cast<size_t>(p.tiles) * 4 + 255) / 256 * 256;
+    p.count_bytes = kCountRegion;
+    p.ok = static_cast<size_t>(p.tiles) * 4 <= kCountRegion;
     const int smem_budget = 232448 - 1024 - 1024 - skinny_stage_bytes_y(p.mp);  // minus slack, static data, Y staging
-    int st = smem_budget / skinny_stage_bytes(p.mp);
+    int st = smem_budget / (fused ? skinny_stage_bytes_fused(p.mp) : skinny_stage_bytes(p.mp));
     p.stages = st > kSkinnyMaxStages ? kSkinnyMaxStages : st;
     return p;
 }
 
-macaq_status run_skinny(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K, const uint8_t *Wq,
-                        const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace, size_t ws_bytes,
-                        int sms, cudaStream_t st) {
-    const SkinnyPlan p = skinny_plan(M, N, K, sms);
+// The skinny GEMM. fused_b = 0: A is Xq/Asf (quantized activations). fused_b > 0: A is bf16 X
+// (M <= 16) and the kernel applies 1/s (inv_s, may be null), H_b and MXFP4 itself.
+template <int kFusedB>
+macaq_status launch_skinny(const CUtensorMap &wmap, const CUtensorMap &xmap, const CUtensorMap &sfwmap,
+                           const CUtensorMap &sfxmap, const CUtensorMap &ymap, const SkinnyArgs &g, const SkinnyPlan &p,
+                           cudaStream_t st) {
+    const int sb = kFusedB > 0 ? skinny_stage_bytes_fused(p.mp) : skinny_stage_bytes(p.mp);
+    const size_t smem = 1024 + static_cast<size_t>(p.stages) * sb + skinny_stage_bytes_y(p.mp);
+    macaq_status s = set_smem(gemm_mxf4_skinny_kernel<kFusedB>, smem);
+    if (s != MACAQ_OK) return s;
+    gemm_mxf4_skinny_kernel<kFusedB><<<p.ctas, kFusedB > 0 ? 320 : 192, smem, st>>>(wmap, xmap, sfwmap, sfxmap, ymap, g);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+}
+
+macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, int32_t fused_b, int64_t M, int64_t N,
+                        int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
+                        size_t ws_bytes, int sms, cudaStream_t st) {
+    const bool fused = fused_b > 0;
+    const SkinnyPlan p = skinny_plan(M, N, K, sms, fused);
+    if (!p.ok) return MACAQ_ERR_SHAPE;
     if (ws_bytes < p.partial_bytes + p.count_bytes) return MACAQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MACAQ_ERR_ALIGNMENT;
     CUtensorMap wmap, xmap, sfwmap, sfxmap, ymap;
     macaq_status s = tensor_map_2d(&wmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128,
                                    CU_TENSOR_MAP_SWIZZLE_128B);
-    if (s == MACAQ_OK)
-        s = tensor_map_2d(&xmap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, kBKBytes, p.mp,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s == MACAQ_OK) {
+        if (fused)  // bf16 X, one K-block (256 elements) of all 16 rows per box; rows past M read as zero
+            s = tensor_map_2d(&xmap, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 256, p.mp,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+        else
+            s = tensor_map_2d(&xmap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, kBKBytes, p.mp,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     // replicated scale factors: (128 B, the K-block's two tiles, 8-row group, replica (stride 0), tile)
     const uint32_t sbox[5] = {128, 2, 4, 4, 1};
     const uint64_t sstr[4] = {512, 128, 0, 512};
@@ -306,8 +334,12 @@ macaq_status run_skinny(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t
         s = tensor_map(&sfwmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, d, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (s == MACAQ_OK) {
-        const uint64_t d[5] = {128, 2, 4, 4, macaq_sf_bytes(M, K) / 512};
-        s = tensor_map(&sfxmap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, d, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (fused) {
+            sfxmap = sfwmap;  // unused: the kernel writes X's scale factors itself
+        } else {
+            const uint64_t d[5] = {128, 2, 4, 4, macaq_sf_bytes(M, K) / 512};
+            s = tensor_map(&sfxmap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, d, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE);
+        }
     }
     // Y as bf16 [M, N]; each epilogue warp stores a 32-column x Mp-row box
     if (s == MACAQ_OK)
@@ -327,12 +359,16 @@ macaq_status run_skinny(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t
     g.units = p.units;
     g.gran = p.gran;
     g.wait_limit_ns = g_wait_limit_ns.load();
-    const size_t smem = 1024 + static_cast<size_t>(p.stages) * skinny_stage_bytes(p.mp) + skinny_stage_bytes_y(p.mp);
-    s = set_smem(gemm_mxf4_skinny_kernel, smem);
-    if (s != MACAQ_OK) return s;
-    gemm_mxf4_skinny_kernel<<<p.ctas, 192, smem, st>>>(wmap, xmap, sfwmap, sfxmap, ymap, g);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+    g.inv_s = inv_s;
+    switch (fused_b) {
+        case 0: return launch_skinny<0>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
+        case 1: return launch_skinny<1>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
+        case 16: return launch_skinny<16>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
+        case 32: return launch_skinny<32>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
+        case 64: return launch_skinny<64>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
+        case 128: return launch_skinny<128>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
+        default: return MACAQ_ERR_UNSUPPORTED;
+    }
 }
 
 macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, int32_t E, int64_t rows, int64_t N,
@@ -352,8 +388,9 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
     macaq_status s = device_info(&dev);
     if (s != MACAQ_OK) return s;
 
-    if (offsets == nullptr && rows <= kSkinnyMaxM && K % 256 == 0 && workspace != nullptr)
-        return run_skinny(A, Asf, rows, N, K, Wq, Wsf, Y, out_dtype, workspace, ws_bytes, dev.sms, st);
+    if (offsets == nullptr && rows <= kSkinnyMaxM && K % 256 == 0 && workspace != nullptr &&
+        skinny_plan(rows, N, K, dev.sms).ok)
+        return run_skinny(A, Asf, nullptr, 0, rows, N, K, Wq, Wsf, Y, out_dtype, workspace, ws_bytes, dev.sms, st);
 
     const int BN = (N % 256 == 0) ? 256 : 128;
     const bool grouped = offsets != nullptr;
@@ -494,10 +531,68 @@ macaq_status linear_fixed_scratch(const uint8_t *A, const uint8_t *Asf, int64_t 
     s = device_info(&dev);
     if (s != MACAQ_OK) return s;
     const SkinnyPlan p = skinny_plan(M, N, K, dev.sms);
+    if (!p.ok) return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, nullptr, 0, st);
     if (p.partial_bytes + p.count_bytes > MACAQ_FIXED_SCRATCH_BYTES) return MACAQ_ERR_WORKSPACE;
-    const cudaError_t e = cudaMemsetAsync(scratch, 0, p.count_bytes, st);  // the per-tile counters
+    const size_t used_counts = (static_cast<size_t>(p.tiles) * 4 + 255) / 256 * 256;
+    const cudaError_t e = cudaMemsetAsync(scratch, 0, used_counts, st);  // the per-tile counters this call uses
     if (e != cudaSuccess) return cuda_fail(e);
     return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, scratch, MACAQ_FIXED_SCRATCH_BYTES, st);
+}
+
+// ------------------------------------------------------------------------ fused layer (a7)
+// Workspace of the fused layer: the GEMM's own region (skinny counters and partials, when the skinny
+// kernel runs), then room for the quantized activations and their scale factors, which the two-kernel
+// form writes and reads back. Offsets are 256-byte aligned.
+struct FusedLayout {
+    size_t gemm_ws, a_off, sf_off, total;
+    bool in_kernel;   // the skinny kernel quantizes X itself
+};
+
+FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
+    FusedLayout f{};
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    if (E == 0 && M >= 1 && M <= kSkinnyMaxM && K % 256 == 0) {
+        const SkinnyPlan p = skinny_plan(M, N, K, sms, M <= kSkinnyFusedMaxM);
+        if (p.ok) {
+            f.gemm_ws = up(p.count_bytes + p.partial_bytes);
+            f.in_kernel = M <= kSkinnyFusedMaxM;
+        }
+    }
+    f.a_off = f.gemm_ws;
+    f.sf_off = f.a_off + up(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
+    f.total = f.sf_off + (E > 0 ? macaq_grouped_sf_bytes(M, E, K) : macaq_sf_bytes(M, K));
+    return f;
+}
+
+// Y = (X diag(1/s) H_b, MXFP4) x W'^T from bf16 X. Dense calls with M <= 16 and K % 256 == 0 run the
+// skinny kernel with its quantizer warps: no quantized activation touches HBM. Every other shape (and
+// every grouped call) quantizes X into the workspace and runs the GEMM on it, two launches in stream
+// order: re-quantizing an A tile for every output tile it meets would cost more than the
+// 0.53125 B/element round trip once M is large.
+macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const int32_t *offsets, int32_t E, int64_t M,
+                          int64_t N, int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype,
+                          void *workspace, size_t ws_bytes, cudaStream_t st) {
+    if (M < 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 128 != 0) return MACAQ_ERR_SHAPE;
+    if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
+    if (offsets != nullptr && (E < 1 || E > 1024)) return MACAQ_ERR_SHAPE;
+    if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
+    if (M == 0) return MACAQ_OK;
+    if (X == nullptr || Wq == nullptr || Wsf == nullptr || Y == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(Y) ||
+        !aligned16(workspace) || !aligned16(offsets))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+    const FusedLayout f = fused_layout(M, N, K, offsets != nullptr ? E : 0, dev.sms);
+    if (workspace == nullptr || ws_bytes < f.total) return MACAQ_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (offsets == nullptr && f.in_kernel)
+        return run_skinny(X, nullptr, inv_s, b, M, N, K, Wq, Wsf, Y, out_dtype, ws, f.gemm_ws, dev.sms, st);
+    s = quantize(X, inv_s, M, K, b, false, offsets, offsets != nullptr ? E : 0, ws + f.a_off, ws + f.sf_off, nullptr, st);
+    if (s != MACAQ_OK) return s;
+    return gemm(ws + f.a_off, ws + f.sf_off, offsets, offsets != nullptr ? E : 1, M, N, K, Wq, Wsf, Y, out_dtype,
+                f.gemm_ws > 0 ? ws : nullptr, f.gemm_ws, st);
 }
 
 }  // namespace macaq
@@ -537,7 +632,15 @@ size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E) {
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 0;
     const macaq::SkinnyPlan p = macaq::skinny_plan(M, N, K, sms);
-    return p.partial_bytes + p.count_bytes;
+    return p.ok ? p.partial_bytes + p.count_bytes : 0;
+}
+
+size_t macaq_fused_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E) {
+    if (M < 0 || N <= 0 || N % 128 != 0 || K <= 0 || K % 128 != 0 || E < 0) return 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return macaq::fused_layout(M, N, K, E, sms).total;
 }
 
 macaq_status macaq_prep_weights(const void *W, const float *s, int64_t N, int64_t K, int32_t had_block, uint8_t *Wq,
@@ -557,8 +660,9 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
 macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M, int64_t N,
                           int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
                           int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
-    (void)inv_s, (void)had_block;
-    if (mode == MACAQ_A_BF16_FUSED) return MACAQ_ERR_UNSUPPORTED;
+    if (mode == MACAQ_A_BF16_FUSED)
+        return macaq::linear_fused(A, inv_s, had_block, nullptr, 0, M, N, K, Wq, Wsf, Y, out_dtype, workspace, ws_bytes,
+                                   static_cast<cudaStream_t>(stream));
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
     return macaq::gemm(static_cast<const uint8_t *>(A), Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, workspace,
                        ws_bytes, static_cast<cudaStream_t>(stream));
@@ -578,9 +682,11 @@ macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *As
                                   const int32_t *group_offsets, int32_t E, int64_t total_rows, int64_t N, int64_t K,
                                   int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
                                   int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
-    (void)inv_s, (void)had_block, (void)workspace, (void)ws_bytes;
-    if (mode != MACAQ_A_QUANTIZED) return mode == MACAQ_A_BF16_FUSED ? MACAQ_ERR_UNSUPPORTED : MACAQ_ERR_INVALID_ARG;
     if (group_offsets == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (mode == MACAQ_A_BF16_FUSED)
+        return macaq::linear_fused(A, inv_s, had_block, group_offsets, E, total_rows, N, K, Wq, Wsf, Y, out_dtype,
+                                   workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
     return macaq::gemm(static_cast<const uint8_t *>(A), Asf, group_offsets, E, total_rows, N, K, Wq, Wsf, Y,
                        out_dtype, nullptr, 0, static_cast<cudaStream_t>(stream));
 }

@@ -98,6 +98,59 @@ __device__ __forceinline__ void load_mul(const float *mul, uint64_t (&mv)[16]) {
     }
 }
 
+// Hadamard stages (and, for weights, the exact 1/b) on one 32-element group held as 16 packed fp32
+// pairs, then its MXFP4 encoding: the 16 code bytes (even k in the low nibble) and the E8M0
+// exponent. For b >= 64 the group is paired with the groups of lanes lane ^ 1 (and lane ^ 2), which
+// hold the next groups of the same row: the whole warp calls it together.
+template <int kB, bool kWeight>
+__device__ __forceinline__ void transform_quantize_group(uint64_t (&p)[16], uint4 &packed, uint32_t &E8) {
+    if constexpr (kB > 1) {
+        fwht_in_thread<kB>(p);
+        if constexpr (kB >= 64) fwht_cross_lane(p, 1);
+        if constexpr (kB >= 128) fwht_cross_lane(p, 2);
+        if constexpr (kWeight) {
+            const uint64_t inv_b = pk2(1.0f / kB, 1.0f / kB);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], inv_b);
+        }
+    }
+
+    float mx[16];  // max |v| as a tree: short dependency chains
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float lo, hi;
+        upk2(p[i], lo, hi);
+        mx[i] = fmaxf(fabsf(lo), fabsf(hi));
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+    const int ef = static_cast<int>(__float_as_uint(mx[0]) >> 23);  // biased exponent (amax >= 0)
+    E8 = static_cast<uint32_t>(ef > 2 ? ef - 2 : 0);
+    const float inv_scale = __uint_as_float((254u - E8) << 23);     // 2^(127 - E), a normal float
+    const uint64_t inv_scale2 = pk2(inv_scale, inv_scale);
+
+    float y[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) upk2(mul2(p[i], inv_scale2), y[2 * i], y[2 * i + 1]);
+    packed.x = cvt_e2m1x8(y + 0);
+    packed.y = cvt_e2m1x8(y + 8);
+    packed.z = cvt_e2m1x8(y + 16);
+    packed.w = cvt_e2m1x8(y + 24);
+}
+
+// Unpacks 32 bf16 (four 16-byte words, element order) into 16 packed fp32 pairs.
+__device__ __forceinline__ void unpack_bf16x32(const uint4 (&raw)[4], uint64_t (&p)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        p[4 * i + 0] = pk2(__uint_as_float(raw[i].x << 16), __uint_as_float(raw[i].x & 0xFFFF0000u));
+        p[4 * i + 1] = pk2(__uint_as_float(raw[i].y << 16), __uint_as_float(raw[i].y & 0xFFFF0000u));
+        p[4 * i + 2] = pk2(__uint_as_float(raw[i].z << 16), __uint_as_float(raw[i].z & 0xFFFF0000u));
+        p[4 * i + 3] = pk2(__uint_as_float(raw[i].w << 16), __uint_as_float(raw[i].w & 0xFFFF0000u));
+    }
+}
+
 // Work split: the K axis is cut into column slabs of slab_groups groups; a tile is tile_rows rows of
 // one slab (always 256 groups, 16 KB). A CTA keeps one slab for its whole life and walks its row
 // tiles, so each consumer thread owns one fixed group column and keeps that column's 32 multipliers
@@ -173,13 +226,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
                 raw[i] = *reinterpret_cast<const uint4 *>(lp + phys * 16);
             }
             uint64_t p[16];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                p[4 * i + 0] = pk2(__uint_as_float(raw[i].x << 16), __uint_as_float(raw[i].x & 0xFFFF0000u));
-                p[4 * i + 1] = pk2(__uint_as_float(raw[i].y << 16), __uint_as_float(raw[i].y & 0xFFFF0000u));
-                p[4 * i + 2] = pk2(__uint_as_float(raw[i].z << 16), __uint_as_float(raw[i].z & 0xFFFF0000u));
-                p[4 * i + 3] = pk2(__uint_as_float(raw[i].w << 16), __uint_as_float(raw[i].w & 0xFFFF0000u));
-            }
+            unpack_bf16x32(raw, p);
             // Release the stage only after every lane has its words in registers (the unpacking above
             // consumed them), and order those generic-proxy reads before the next TMA write of the
             // stage, which is an async-proxy access.
@@ -191,41 +238,9 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
                 for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
             }
 
-            if constexpr (kB > 1) {
-                fwht_in_thread<kB>(p);
-                if constexpr (kB >= 64) fwht_cross_lane(p, 1);
-                if constexpr (kB >= 128) fwht_cross_lane(p, 2);
-                if constexpr (kWeight) {
-                    const uint64_t inv_b = pk2(1.0f / kB, 1.0f / kB);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], inv_b);
-                }
-            }
-
-            float mx[16];  // max |v| as a tree: short dependency chains
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float lo, hi;
-                upk2(p[i], lo, hi);
-                mx[i] = fmaxf(fabsf(lo), fabsf(hi));
-            }
-#pragma unroll
-            for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-                for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-            const int ef = static_cast<int>(__float_as_uint(mx[0]) >> 23);  // biased exponent (amax >= 0)
-            const uint32_t E8 = static_cast<uint32_t>(ef > 2 ? ef - 2 : 0);
-            const float inv_scale = __uint_as_float((254u - E8) << 23);     // 2^(127 - E), a normal float
-            const uint64_t inv_scale2 = pk2(inv_scale, inv_scale);
-
-            float y[32];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) upk2(mul2(p[i], inv_scale2), y[2 * i], y[2 * i + 1]);
             uint4 packed;
-            packed.x = cvt_e2m1x8(y + 0);
-            packed.y = cvt_e2m1x8(y + 8);
-            packed.z = cvt_e2m1x8(y + 16);
-            packed.w = cvt_e2m1x8(y + 24);
+            uint32_t E8;
+            transform_quantize_group<kB, kWeight>(p, packed, E8);
             const bool store = e >= 0;
             if (store)
                 *reinterpret_cast<uint4 *>(a.q + static_cast<uint64_t>(m) * (a.K / 2) + g * 16) = packed;
