@@ -244,6 +244,7 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    griddep_wait();  // the operands and Y may belong to the previous kernel in the stream
     load_group_layout(kGrouped ? g.offsets : nullptr, kGrouped ? g.E : 1, g.rows, s_off, s_tb);  // block-wide
     const uint32_t m_tiles = static_cast<uint32_t>(s_tb[kGrouped ? g.E : 1]);
     const uint32_t n_tiles = static_cast<uint32_t>(g.N / BN);
@@ -269,6 +270,7 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    griddep_launch_dependents();
     const uint32_t tmem = tmem_slot;
 
     const int K = g.K;
@@ -497,6 +499,8 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     tc_fence_before();
     cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
     tc_fence_after();
+    griddep_wait();  // the operands and Y may belong to the previous kernel in the stream
+    griddep_launch_dependents();
     const uint32_t tmem = tmem_slot;
     const uint32_t leader_failed_addr = map_to_rank(smem_u32(const_cast<int *>(&failed)), 0);
 
@@ -739,33 +743,45 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    griddep_launch_dependents();
     const uint32_t tmem = tmem_slot;                 // accumulators at columns 0 and 128
     const uint32_t t_sfw = tmem + 256, t_sfx = tmem + 264;
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ TMA producer
-            uint32_t j = 0;
-            for (uint32_t u = u_begin; u < u_end; ++u, ++j) {
+            // The weights do not depend on the previous kernel in the stream: the first S stages' W'
+            // tiles and scale factors are requested before waiting for it; the activations after.
+            auto load_w = [&](uint32_t u, int s) {
                 const uint32_t tile = u / num_kb;
                 const int kb = static_cast<int>(u - tile * num_kb);
-                const int s = j % S;
-                if (j >= static_cast<uint32_t>(S) && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) break;
+                if constexpr (kFused) mbar_arrive_expect_tx(&full_bar[s], 128 * kBKBytes + 4096);
+                else mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
+                tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
+                tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
+            };
+            auto load_x = [&](uint32_t u, int s) {
+                const int kb = static_cast<int>(u % num_kb);
                 if constexpr (kFused) {
-                    mbar_arrive_expect_tx(&full_bar[s], 128 * kBKBytes + 4096);
-                    tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
-                    tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
                     // X's K-block as bf16 (rows past M read as zero) and its 256 multipliers
                     mbar_arrive_expect_tx(&xin_bar[s], mp * 512 + (g.inv_s != nullptr ? 1024 : 0));
                     tma_load_2d(sXin(s), &xmap, &xin_bar[s], kb * 256, 0);
                     if (g.inv_s != nullptr) bulk_load(sInv(s), g.inv_s + kb * 256, 1024, &xin_bar[s]);
                 } else {
-                    mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
-                    tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
                     tma_load_2d(sX(s), &xmap, &full_bar[s], kb * kBKBytes, 0);
-                    tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
                     tma_load_5d(sSfx(s), &sfxmap, &full_bar[s], 0, 0, 0, 0, 2 * kb);
                 }
+            };
+            const uint32_t pre = min(static_cast<uint32_t>(S), u_end > u_begin ? u_end - u_begin : 0u);
+            for (uint32_t i = 0; i < pre; ++i) load_w(u_begin + i, static_cast<int>(i));
+            griddep_wait();
+            for (uint32_t i = 0; i < pre; ++i) load_x(u_begin + i, static_cast<int>(i));
+            uint32_t j = pre;
+            for (uint32_t u = u_begin + pre; u < u_end; ++u, ++j) {
+                const int s = j % S;
+                if (!mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) break;
+                load_w(u, s);
+                load_x(u, s);
             }
             for (uint32_t i = (j > static_cast<uint32_t>(S) ? j - S : 0); i < j; ++i)
                 if (!mbar_wait(&full_bar[i % S], (i / S) & 1, kDrainLimitNs)) break;

@@ -153,6 +153,34 @@ macaq_status set_smem(Kernel k, size_t bytes) {
     return MACAQ_OK;
 }
 
+// Every kernel is launched with programmatic stream serialization: it may start its prologue while
+// the previous kernel in the stream finishes, and waits for that kernel (griddep_wait) before it
+// touches memory the previous kernel may own. cluster > 1 adds the cluster shape.
+template <typename Kernel, typename... Args>
+macaq_status launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, unsigned cluster, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    unsigned n = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------------------------ quantization
 template <int kB, bool kWeight>
 macaq_status run_quant_b(const CUtensorMap &map, const QuantArgs &a, int grid, cudaStream_t st) {
@@ -160,9 +188,7 @@ macaq_status run_quant_b(const CUtensorMap &map, const QuantArgs &a, int grid, c
     const size_t smem = quant_smem_bytes(a.E);
     macaq_status s = set_smem(k, smem);
     if (s != MACAQ_OK) return s;
-    k<<<grid, kQThreads, smem, st>>>(map, a);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+    return launch(k, dim3(grid), dim3(kQThreads), smem, st, 1, map, a);
 }
 
 template <bool kWeight>
@@ -235,9 +261,7 @@ macaq_status run_gemm(const CUtensorMap &amap, const CUtensorMap &bmap, const Ge
     const size_t smem = gemm_smem_bytes<BN>(kGrouped ? g.E : 0);
     macaq_status s = set_smem(k, smem);
     if (s != MACAQ_OK) return s;
-    k<<<grid, kGemmThreads, smem, st>>>(amap, bmap, g);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+    return launch(k, grid, dim3(kGemmThreads), smem, st, 1, amap, bmap, g);
 }
 
 // ------------------------------------------------------------------------ skinny GEMM (M <= 128)
@@ -302,9 +326,8 @@ macaq_status launch_skinny(const CUtensorMap &wmap, const CUtensorMap &xmap, con
     const size_t smem = 1024 + static_cast<size_t>(p.stages) * sb + skinny_stage_bytes_y(p.mp);
     macaq_status s = set_smem(gemm_mxf4_skinny_kernel<kFusedB>, smem);
     if (s != MACAQ_OK) return s;
-    gemm_mxf4_skinny_kernel<kFusedB><<<p.ctas, kFusedB > 0 ? 320 : 192, smem, st>>>(wmap, xmap, sfwmap, sfxmap, ymap, g);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+    return launch(gemm_mxf4_skinny_kernel<kFusedB>, dim3(p.ctas), dim3(kFusedB > 0 ? 320 : 192), smem, st, 1, wmap, xmap,
+                  sfwmap, sfxmap, ymap, g);
 }
 
 macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, int32_t fused_b, int64_t M, int64_t N,
@@ -455,22 +478,8 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
         const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
         s = set_smem(gemm_mxf4_pair_kernel, PairCfg::kSmemBytes);
         if (s != MACAQ_OK) return s;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * pairs);
-        cfg.blockDim = dim3(PairCfg::kThreads);
-        cfg.dynamicSmemBytes = PairCfg::kSmemBytes;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_mxf4_pair_kernel, amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes);
-        if (e != cudaSuccess) return cuda_fail(e);
-        e = cudaGetLastError();
-        return e == cudaSuccess ? MACAQ_OK : cuda_fail(e);
+        return launch(gemm_mxf4_pair_kernel, dim3(2 * pairs), dim3(PairCfg::kThreads), PairCfg::kSmemBytes, st, 2, amap,
+                      bmap, sfamap, sfbmap, ymap, g, replica_boxes);
     }
 
     CUtensorMap amap, bmap;

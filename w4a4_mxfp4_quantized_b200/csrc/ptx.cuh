@@ -70,6 +70,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
+// ------------------------------------------------------------------------------------ dependent launch
+// Programmatic dependent launch. griddep_wait: wait until the grids this one depends on (the previous
+// kernel in the stream, when it was launched with the attribute) have completed and their memory is
+// visible; without such a dependency it returns at once. griddep_launch_dependents: once every CTA of
+// this grid has executed it (or exited), the next grid may start its prologue.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------ TMA
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -180,7 +180,9 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
         fence_mbar_init();
         if (first_tile < a.row_tiles) prefetch_tensor_map(&xmap);
     }
+    griddep_wait();  // X, the offsets and the outputs may belong to the previous kernel in the stream
     load_group_layout(a.offsets, a.E, a.rows, s_off, s_tb);  // contains __syncthreads
+    griddep_launch_dependents();
 
     if (warp == kQConsumerWarps) {
         // ---------------------------------------------------------------- producer
