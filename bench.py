@@ -130,6 +130,20 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ------------------------------------------------------------------------------------ ranks
+def max_over_ranks(ms: float, dist_on: bool, device) -> float:
+    """The slowest rank's time: every rank runs its own replica, the job ends with the last one."""
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank does flops_per_step per step, the step takes ms_per_step."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------------------------ our arm
 def make_layer(M, dev, copies, plain=False):
     """The layer's device buffers. plain=True is the plain-MXFP4 comparator: no per-channel scale
@@ -170,6 +184,9 @@ def copies_for(M):
 
 
 def run_layer(mq, L, i, parts=("aq", "gemm")):
+    if "fused" in parts:  # the layer in one call from bf16 X (quantizer inside the GEMM for M <= 16)
+        mq.linear(L["X"][i], None, L["Wq"][i], L["Wsf"][i], mode=mq.A_BF16_FUSED, inv_s=L["inv_s"],
+                  had_block=L["b"], Y=L["Y"][i])
     if "aq" in parts:
         mq.act_quant(L["X"][i], L["inv_s"], L["b"], Xq=L["Xq"][i], Xsf=L["Xsf"][i])
     if "gemm" in parts:
@@ -195,14 +212,15 @@ def replay_ms(g, stream):
     return a.elapsed_time(b)
 
 
-def time_layer(M, steps, warmup, dev, dist_on, plain=False):
-    """Device time of `steps` layer passes (graph replay, rotating copies) and of each kernel alone."""
+def time_layer(M, steps, warmup, dev, dist_on, plain=False, fused=False):
+    """Device time of `steps` layer passes (graph replay, rotating copies) and of each kernel alone.
+    fused=True also times the one-call fused layer (returned as L["fused_ms"], per pass)."""
     import w4a4_mxfp4_quantized_b200 as mq
 
     ncopy = copies_for(M)
     L = make_layer(M, dev, ncopy, plain)
     for i in range(max(warmup, 1)):
-        run_layer(mq, L, i % ncopy)
+        run_layer(mq, L, i % ncopy, ("aq", "gemm", "fused") if fused else ("aq", "gemm"))
     torch.cuda.synchronize(dev)
     g_pair = capture(mq, L, steps, ncopy, ("aq", "gemm"))
     g_aq = capture(mq, L, steps, ncopy, ("aq",))
@@ -224,6 +242,11 @@ def time_layer(M, steps, warmup, dev, dist_on, plain=False):
         torch.distributed.barrier()
     aq_ms = replay_ms(g_aq, stream) / steps
     gemm_ms = replay_ms(g_gemm, stream) / steps
+    if fused:
+        g_fused = capture(mq, L, steps, ncopy, ("fused",))
+        g_fused.replay()
+        L["fused_ms"] = replay_ms(g_fused, stream) / steps
+        del g_fused
     status = mq.device_status()
     assert status == 0, f"device status {status}"
     del g_pair, g_aq, g_gemm
@@ -337,11 +360,8 @@ def main():
     with ClockSampler(local) as clk:
         total_ms, aq_ms, gemm_ms, L = time_layer(M, args.steps, args.warmup, dev, dist_on)
     clocks = clk.summary()
-    t = torch.tensor([total_ms], device=dev)
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_step = t.item() / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    ms_step = max_over_ranks(total_ms, dist_on, dev) / args.steps
+    value = job_tflops(world, flops, ms_step)
 
     del L
     p_total, p_aq, p_gemm, _ = time_layer(M, args.steps, args.warmup, dev, dist_on, plain=True)
@@ -351,7 +371,8 @@ def main():
                 "pages_figure_for_context": "2.3% end-to-end, Qwen3-32B in vLLM, hardware not stated"}
     _, _, _, L = time_layer(M, 3, 1, dev, dist_on)
     e2e_ms, h2d, d2h = time_e2e(M, max(3, args.steps // 2), 2, dev, L)
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist_on, dev)
+    e2e_value = job_tflops(world, flops, e2e_ms)
 
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     gemm_kernel = gemm_kernel_name(M)
@@ -359,7 +380,9 @@ def main():
     sweep = []
     if not args.no_sweep:
         for m in M_SWEEP:
-            tot, aq, gm, _ = time_layer(m, max(10, args.steps), args.warmup, dev, dist_on)
+            tot, aq, gm, Lm = time_layer(m, max(10, args.steps), args.warmup, dev, dist_on, fused=True)
+            fz = Lm["fused_ms"]
+            del Lm
             fl = 2.0 * m * N_DIM * K_DIM
             g_bytes = N_DIM * K_DIM * 0.53125 + m * K_DIM * 0.53125 + m * N_DIM * 2
             a_bytes = m * K_DIM * (2 + 0.5 + 1 / 32)
@@ -369,7 +392,11 @@ def main():
                           "gemm_frac_fp4_peak": fl / (gm * 1e-3) / 1e12 / fp4_peak,
                           "gemm_frac_hbm": g_bytes / (gm * 1e-3) / 1e9 / hbm,
                           "act_quant_us": aq * 1e3, "act_quant_gbs": a_bytes / (aq * 1e-3) / 1e9,
-                          "act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm})
+                          "act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm,
+                          "fused_layer_us": fz * 1e3,
+                          "fused_layer_tflops": fl / (fz * 1e-3) / 1e12,
+                          "fused_form": "quantizer warps inside the skinny GEMM" if m <= 16
+                          else "quantizer pass + GEMM in one call"})
     if rank != 0:
         if dist_on:
             torch.distributed.destroy_process_group()

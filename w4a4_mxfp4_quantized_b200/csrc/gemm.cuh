@@ -475,6 +475,13 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     const int kq = K / 128;
     const int num_kb = K / 256;
     const uint64_t limit = g.wait_limit_ns;
+    // The pair's tiles: cluster, cluster + clusters, ... (tile t, all K-blocks [0, num_kb)).
+    auto segment = [&](uint32_t i, uint32_t &t, int &k0, int &k1) -> bool {
+        t = cluster + i * clusters;
+        k0 = 0;
+        k1 = num_kb;
+        return t < num_tiles;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -511,14 +518,16 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
             const bool sf = warp == 10;
             uint32_t j = 0;
             bool stop = false;
-            for (uint32_t t = cluster; t < num_tiles && !stop; t += clusters) {
+            uint32_t t;
+            int k0, k1;
+            for (uint32_t sgi = 0; !stop && segment(sgi, t, k0, k1); ++sgi) {
                 uint32_t mt, nt;
                 raster(t, m_tiles, n_tiles, mt, nt);
                 const int32_t arow = static_cast<int32_t>(mt * 256 + rank * 128);
                 const int32_t brow = static_cast<int32_t>(nt * 256 + rank * 128);
                 const int32_t a_tile = static_cast<int32_t>((mt * 2 + rank) * kq);   // first 128x4 tile of A's rows
                 const int32_t b_tile = static_cast<int32_t>(nt * 2 * kq);            // of B's first 128 rows
-                for (int kb = 0; kb < num_kb; ++kb, ++j) {
+                for (int kb = k0; kb < k1; ++kb, ++j) {
                     const int s = j % S;
                     if (j >= S && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) {
                         stop = true;
@@ -559,13 +568,15 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
             uint32_t j = 0;
             uint32_t tiles_done = 0;
             bool stop = false;
-            for (uint32_t t = cluster; t < num_tiles && !stop; t += clusters, ++tiles_done) {
+            uint32_t t;
+            int k0, k1;
+            for (uint32_t sgi = 0; !stop && segment(sgi, t, k0, k1); ++sgi, ++tiles_done) {
                 if (tiles_done > 0 && !mbar_wait_or_abort(&accum_empty, (tiles_done - 1) & 1, limit, &failed)) {
                     stop = true;
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < num_kb; ++kb, ++j) {
+                for (int kb = k0; kb < k1; ++kb, ++j) {
                     const int s = j % S;
                     if (!mbar_wait_or_abort(&full_bar[s], (j / S) & 1, limit, &failed)) {
                         stop = true;
@@ -582,7 +593,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
                     for (int q = 0; q < 4; ++q) {
                         const int c = q >> 1;
                         tc_mma_mxf4_pair(tmem, adesc + 2 * q, bdesc + 2 * q, (q & 1) ? idesc_hi : idesc_lo,
-                                         tmem + C::kTmemSfa + 4 * c, tmem + C::kTmemSfb + c * 8, (kb | q) != 0 ? 1u : 0u);
+                                         tmem + C::kTmemSfa + 4 * c, tmem + C::kTmemSfb + c * 8, (kb != k0 || q != 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&empty_bar[s]);
                 }
@@ -598,7 +609,9 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const uint32_t empty_addr = map_to_rank(smem_u32(&accum_empty), 0);
         uint32_t tiles_done = 0;
-        for (uint32_t t = cluster; t < num_tiles; t += clusters, ++tiles_done) {
+        uint32_t t;
+        int k0, k1;
+        for (uint32_t sgi = 0; segment(sgi, t, k0, k1); ++sgi, ++tiles_done) {
             uint32_t mt, nt;
             raster(t, m_tiles, n_tiles, mt, nt);
             if (!mbar_wait_or_abort(&accum_full, tiles_done & 1, limit, &failed)) break;
@@ -644,7 +657,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
 // activation ever goes to HBM. Source: the aipolix.com page, paragraph 2 (transform on each layer's
 // activations at inference); glonce.com page, paragraph 5 (W4A4 dense matmul).
 constexpr int kSkinnyMaxStages = 12;
-constexpr int kSkinnyFusedMaxM = 16;
+constexpr int kSkinnyFusedMaxM = 4;
 
 struct SkinnyArgs {
     void *y;                   // [M, N]
@@ -712,7 +725,7 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], kFused ? 5 : 1);   // fused: the producer and the four quantizer warps
+            mbar_init(&full_bar[s], kFused ? 2 : 1);   // fused: the producer and the stage's quantizer warp
             mbar_init(&empty_bar[s], 1);
             mbar_init(&xin_bar[s], 1);
         }
@@ -733,11 +746,14 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
         tmem_relinquish();
     }
     if constexpr (kFused) {
-        // the quantizer writes only the scale bytes of rows < 16; the rest of each replicated block
-        // stays zero for the whole launch
-        for (int s = 0; s < S; ++s)
+        // the quantizer writes only the codes and scale bytes of rows < M; the rest of the X operand
+        // and of each replicated scale block stays zero for the whole launch
+        for (int s = 0; s < S; ++s) {
             for (int i = threadIdx.x; i < 4096 / 16; i += blockDim.x)
                 reinterpret_cast<uint4 *>(sSfx(s))[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = threadIdx.x; i < mp * kBKBytes / 16; i += blockDim.x)
+                reinterpret_cast<uint4 *>(sX(s))[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
         fence_proxy_async_smem();
     }
     tc_fence_before();
@@ -825,39 +841,51 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
         }
     } else if (kFused && warp >= 6) {
         // ---------------------------------------------------------------- quantizer (fused form)
-        const int t = threadIdx.x - 192;      // 0..127
-        const int m = t >> 3;                 // activation row (< 16)
-        const int gq = t & 7;                 // 32-element group inside the K-block
-        uint32_t j = 0;
-        for (uint32_t u = u_begin; u < u_end; ++u, ++j) {
+        // Warp 6 + w takes the stages j = w, w + 4, ...: four K-blocks are quantized at once. In a
+        // K-block, group index gi = 8 row + (32-element group); lane l takes gi = l, l + 32, ... over
+        // the M live rows (adjacent lanes hold adjacent groups of one row, as the b >= 64 shuffles
+        // need). Rows M..15 were zeroed once and stay zero.
+        const int qw = warp - 6;
+        const int live = g.M * 8;
+        uint32_t j = qw;
+        for (uint32_t u = u_begin + qw; u < u_end; u += 4, j += 4) {
             const int s = j % S;
             // the whole warp leaves together if any lane's wait ran out (the Hadamard may shuffle)
             if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&xin_bar[s], (j / S) & 1, limit, &failed))) break;
-            const uint8_t *src = sXin(s) + m * 512 + gq * 64;
-            uint4 raw[4];
+            for (int gi0 = 0; gi0 < live; gi0 += 32) {
+                const int gi = gi0 + lane;
+                const int m = gi >> 3;           // row
+                const int gq = gi & 7;           // 32-element group inside the K-block
+                uint4 raw[4] = {};
+                if (gi < live) {
+                    const uint8_t *src = sXin(s) + m * 512 + gq * 64;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) raw[i] = *reinterpret_cast<const uint4 *>(src + i * 16);
-            uint64_t p[16];
-            unpack_bf16x32(raw, p);
-            if (g.inv_s != nullptr) {
-                const float4 *mv4 = reinterpret_cast<const float4 *>(sInv(s) + gq * 128);
+                    for (int i = 0; i < 4; ++i) raw[i] = *reinterpret_cast<const uint4 *>(src + i * 16);
+                }
+                uint64_t p[16];
+                unpack_bf16x32(raw, p);
+                if (g.inv_s != nullptr) {
+                    const float4 *mv4 = reinterpret_cast<const float4 *>(sInv(s) + gq * 128);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 f = mv4[i];
-                    p[2 * i] = mul2(p[2 * i], pk2(f.x, f.y));
-                    p[2 * i + 1] = mul2(p[2 * i + 1], pk2(f.z, f.w));
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 f = mv4[i];
+                        p[2 * i] = mul2(p[2 * i], pk2(f.x, f.y));
+                        p[2 * i + 1] = mul2(p[2 * i + 1], pk2(f.z, f.w));
+                    }
+                }
+                uint4 packed;
+                uint32_t E8;
+                transform_quantize_group<kFusedB, false>(p, packed, E8);
+                if (gi < live) {
+                    // codes: row m's 16-byte chunk gq of the 128-byte row, 128-byte swizzle
+                    *reinterpret_cast<uint4 *>(sX(s) + m * 128 + ((gq ^ (m & 7)) << 4)) = packed;
+                    // exponent: SF tile half gq / 4, column gq % 4, row m (lane m of 32, row quarter 0),
+                    // in each of the four replicas (1 KB apart)
+                    uint8_t *sf = sSfx(s) + ((m >> 3) * 2 + (gq >> 2)) * 128 + (m & 7) * 16 + (gq & 3);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) sf[q * 1024] = static_cast<uint8_t>(E8);
                 }
             }
-            uint4 packed;
-            uint32_t E8;
-            transform_quantize_group<kFusedB, false>(p, packed, E8);
-            // codes: row m's 16-byte chunk gq of the 128-byte row, 128-byte swizzle
-            *reinterpret_cast<uint4 *>(sX(s) + m * 128 + ((gq ^ (m & 7)) << 4)) = packed;
-            // exponent: SF tile half gq / 4, column gq % 4, row m (lane m of 32, row quarter 0), in each
-            // of the four replicas (1 KB apart)
-            uint8_t *sf = sSfx(s) + ((m >> 3) * 2 + (gq >> 2)) * 128 + (m & 7) * 16 + (gq & 3);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) sf[q * 1024] = static_cast<uint8_t>(E8);
             // the stage's input has been read and its operands written: order both before the MMA's
             // (async-proxy) reads and the next TMA write of the stage
             fence_proxy_async_smem();

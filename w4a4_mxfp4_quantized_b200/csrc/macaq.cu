@@ -6,7 +6,9 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <array>
+#include <cmath>
 #include <atomic>
 #include <cstring>
 #include <map>
