@@ -35,6 +35,12 @@ def fused(X, inv, b, Wq, Wsf, out_dtype):
     return mq.linear(X, None, Wq, Wsf, mode=mq.A_BF16_FUSED, inv_s=inv, had_block=b, out_dtype=out_dtype)
 
 
+def counters_zero():
+    """The workspace's counter region stays zero between calls, whatever scratch a call used."""
+    ws = mq._workspace(torch.device("cuda"), 0)
+    return int(ws[:mq.WORKSPACE_COUNTER_BYTES].count_nonzero()) == 0
+
+
 def check_against_oracle(c, b, with_s, Wq_gpu, Wsf_gpu, y32, rows=None):
     """The oracle quantizes X itself; W' comes from the oracle's own weight prep."""
     s = c.s if with_s else None
@@ -76,6 +82,7 @@ def test_two_pass_fusion(M, N, K):
     got = fused(X, inv, b, Wq, Wsf, mq.OUT_F32)
     torch.cuda.synchronize()
     assert torch.equal(got.view(torch.int32), ref.view(torch.int32))
+    assert counters_zero()
     check_against_oracle(c, b, True, Wq, Wsf, got)
 
 
@@ -112,6 +119,13 @@ def test_grouped_fused_equals_two_pass():
     torch.cuda.synchronize()
     rows = np.arange(int(m.offsets[-1]))
     assert torch.equal(got[rows].view(torch.int32), ref[rows].view(torch.int32))
+    assert counters_zero()
+    # a split-tile skinny call on the same workspace right after the grouped fused call
+    c, Wq1, Wsf1, inv1 = layer(31, 64, 1024, 5120, 32, True)
+    X1 = c.X.cuda()
+    assert torch.equal(fused(X1, inv1, 32, Wq1, Wsf1, mq.OUT_F32).view(torch.int32),
+                       unfused(X1, inv1, 32, Wq1, Wsf1, mq.OUT_F32).view(torch.int32))
+    check_against_oracle(c, 32, True, Wq1, Wsf1, unfused(X1, inv1, 32, Wq1, Wsf1, mq.OUT_F32), rows=np.array([0, 63]))
 
 
 def test_fused_needs_a_workspace():

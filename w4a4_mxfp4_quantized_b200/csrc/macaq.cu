@@ -555,7 +555,8 @@ macaq_status linear_fixed_scratch(const uint8_t *A, const uint8_t *Asf, int64_t 
 // kernel runs), then room for the quantized activations and their scale factors, which the two-kernel
 // form writes and reads back. Offsets are 256-byte aligned.
 struct FusedLayout {
-    size_t gemm_ws, a_off, sf_off, total;
+    size_t gemm_ws;   // the skinny kernel's region (counters + partials), 0 when it does not run
+    size_t a_off, sf_off, total;
     bool in_kernel;   // the skinny kernel quantizes X itself
 };
 
@@ -569,7 +570,8 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
             f.in_kernel = M <= kSkinnyFusedMaxM;
         }
     }
-    f.a_off = f.gemm_ws;
+    // the activations never overlap the counter region, whichever kernel runs afterwards
+    f.a_off = std::max(f.gemm_ws, up(kCountRegion));
     f.sf_off = f.a_off + up(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
     f.total = f.sf_off + (E > 0 ? macaq_grouped_sf_bytes(M, E, K) : macaq_sf_bytes(M, K));
     return f;
