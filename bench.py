@@ -253,6 +253,84 @@ def time_layer(M, steps, warmup, dev, dist_on, plain=False, fused=False):
     return total_ms, aq_ms, gemm_ms, L
 
 
+def time_graph(fn, steps, stream):
+    """Device time per call of fn(i), i = 0..steps-1, captured in one graph and replayed."""
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            fn(i)
+    g.replay()
+    ms = replay_ms(g, stream) / steps
+    del g
+    return ms
+
+
+def moe_section(dev, hbm, fp4_peak, steps=20):
+    """The grouped path (MoE 30B-A3B gate/up: 128 experts, top-8 of T tokens, Zipf routing) at
+    T = 64, 1024, 8192: grouped act_quant and grouped GEMM, each timed alone by graph replay.
+    The weights (213 MB prepared) exceed L2 by themselves; X rotates over two copies."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    stream = torch.cuda.current_stream(dev)
+    c0 = inputs.moe_30b_a3b(64, "gate_up")
+    E, N, K = c0.W.shape
+    Wd = c0.W.to(dev)
+    Wq = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
+    Wsf = torch.empty(E, mq.sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    inv = torch.empty(E, K, dtype=torch.float32, device=dev)
+    sd = c0.s.to(dev)
+    for e in range(E):
+        mq.prep_weights(Wd[e], sd[e], HAD_BLOCK, Wq=Wq[e], Wsf=Wsf[e], inv_s=inv[e])
+    del Wd
+    out = []
+    for T in (64, 1024, 8192):
+        c = inputs.moe_30b_a3b(T, "gate_up", draw_w=False)
+        off = c.offsets.to(dev)
+        rows = int(c.offsets[-1])
+        counts = (c.offsets[1:] - c.offsets[:-1]).numpy()
+        Xs = [c.X.to(dev), c.X.to(dev).clone()]
+        Xq = [torch.empty(rows, K // 2, dtype=torch.uint8, device=dev) for _ in range(2)]
+        Xsf = [torch.empty(mq.grouped_sf_bytes(rows, E, K), dtype=torch.uint8, device=dev) for _ in range(2)]
+        Y = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+        aq = time_graph(lambda i: mq.act_quant(Xs[i % 2], inv, HAD_BLOCK, group_offsets=off, Xq=Xq[i % 2],
+                                               Xsf=Xsf[i % 2]), steps, stream)
+        gm = time_graph(lambda i: mq.grouped_linear(Xq[i % 2], Xsf[i % 2], off, Wq, Wsf, Y=Y), steps, stream)
+        assert mq.device_status() == 0
+        flops = 2.0 * N * K * rows
+        g_bytes = int((counts > 0).sum()) * N * K * 0.53125 + rows * (0.53125 * K + 2 * N)
+        a_bytes = rows * K * (2 + 0.5 + 1 / 32)
+        out.append({"T": T, "rows": rows, "experts_used": int((counts > 0).sum()),
+                    "grouped_gemm_us": gm * 1e3, "grouped_gemm_tflops": flops / (gm * 1e-3) / 1e12,
+                    "grouped_gemm_gbs": g_bytes / (gm * 1e-3) / 1e9,
+                    "grouped_gemm_frac_fp4_peak": flops / (gm * 1e-3) / 1e12 / fp4_peak,
+                    "grouped_gemm_frac_hbm": g_bytes / (gm * 1e-3) / 1e9 / hbm,
+                    "grouped_act_quant_us": aq * 1e3, "grouped_act_quant_gbs": a_bytes / (aq * 1e-3) / 1e9,
+                    "grouped_act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm})
+        del Xs, Xq, Xsf, Y
+    return {"workload": f"moe_30b_a3b gate/up E={E} top-8 K={K} N={N} b={HAD_BLOCK}", "points": out}
+
+
+def weight_prep_section(dev, hbm, steps=10):
+    """Offline weight preparation of the Llama-3-8B up/gate weights (bf16 in, codes + SF out)."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    c = inputs.llama3_8b_up(1)
+    W, s = c.W.to(dev), c.s.to(dev)
+    Wq = torch.empty(N_DIM, K_DIM // 2, dtype=torch.uint8, device=dev)
+    Wsf = torch.empty(mq.sf_bytes(N_DIM, K_DIM), dtype=torch.uint8, device=dev)
+    inv = torch.empty(K_DIM, dtype=torch.float32, device=dev)
+    ms = time_graph(lambda i: mq.prep_weights(W, s, HAD_BLOCK, Wq=Wq, Wsf=Wsf, inv_s=inv), steps,
+                    torch.cuda.current_stream(dev))
+    b = N_DIM * K_DIM * (2 + 0.5 + 1 / 32)
+    return {"workload": f"llama3_8b_up_gate W [{N_DIM}, {K_DIM}] b={HAD_BLOCK}", "us": ms * 1e3,
+            "gbs": b / (ms * 1e-3) / 1e9, "frac_hbm": b / (ms * 1e-3) / 1e9 / hbm}
+
+
 def profile_mode(M, steps, warmup, dev):
     """Eager layer passes with no timing: the command the ncu captures run."""
     import w4a4_mxfp4_quantized_b200 as mq
@@ -397,6 +475,8 @@ def main():
                           "fused_layer_tflops": fl / (fz * 1e-3) / 1e12,
                           "fused_form": "quantizer warps inside the skinny GEMM" if m <= 16
                           else "quantizer pass + GEMM in one call"})
+    moe = moe_section(dev, hbm, fp4_peak) if not args.no_sweep else None
+    prep = weight_prep_section(dev, hbm) if not args.no_sweep else None
     if rank != 0:
         if dist_on:
             torch.distributed.destroy_process_group()
@@ -423,6 +503,8 @@ def main():
         "clocks": dict(clocks, window="warm replays (1.5 s of this workload) and the timed replay"),
         "sweep": sweep,
         "transform_overhead": overhead,
+        "moe": moe,
+        "weight_prep": prep,
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
     print(json.dumps(out))
