@@ -645,7 +645,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
 // calls; the partials behind them are written before they are read. When splitting tiles
 // would move more partial bytes than it saves (large M), the ranges are cut on whole tiles instead.
 // Both operands' scale factors arrive replicated (zero-stride TMA view) and go to TMEM with one wide
-// 128x256b copy each per K-block. The stage ring is as deep as shared memory allows; the accumulator
+// 128x256b copy each per K-block. The stage ring has up to kSkinnyMaxStages stages; the accumulator
 // is double-buffered in TMEM. Needs K % 256 == 0.
 //
 // Fused form (kFusedB = Hadamard block b > 0, M <= 16): the activations arrive as bf16 X. Per stage
@@ -656,7 +656,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
 // exponents (four-fold replicated, as the wide copy reads them) straight into the stage. No quantized
 // activation ever goes to HBM. Source: the aipolix.com page, paragraph 2 (transform on each layer's
 // activations at inference); glonce.com page, paragraph 5 (W4A4 dense matmul).
-constexpr int kSkinnyMaxStages = 12;
+constexpr int kSkinnyMaxStages = 4;   // deeper rings measured slower on the decode shapes
 constexpr int kSkinnyFusedMaxM = 4;
 
 struct SkinnyArgs {
