@@ -125,19 +125,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until this thread's bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Waits until this thread's bulk stores are complete.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// Same as tma_load_2d, with an L2 cache-eviction hint (a createpolicy value).
-__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t c0,
-                                                 int32_t c1, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
-        : "memory");
-}
-
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
@@ -145,18 +132,6 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-__device__ __forceinline__ uint64_t policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
 }
 
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05).
@@ -304,23 +279,6 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     return r;
 }
 
-// Unsigned division by a runtime divisor d >= 1 through a multiply-high (n < 2^31):
-// q = (umulhi(n, mul) + n) >> shift with shift = ceil(log2 d), mul = floor(2^32 (2^shift - d) / d) + 1.
-struct FastDiv {
-    uint32_t d, mul, shift;
-};
-
-__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
-    uint32_t s = 0;
-    while ((1ull << s) < d) ++s;
-    const uint64_t m = ((1ull << 32) * ((1ull << s) - d)) / d + 1;
-    return FastDiv{d, static_cast<uint32_t>(m), s};
-}
-
-__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv &f) {
-    return (__umulhi(n, f.mul) + n) >> f.shift;
-}
-
 // ------------------------------------------------------------------------------------ clusters / 2-SM
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -402,11 +360,6 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
         : "memory");
 }
 
-// Scale-factor copy for a 2-SM pair: each CTA's shared-memory block goes to its own TMEM.
-__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 // 2-SM block-scaled MMA: D (+)= A * B^T with A 256 x 64 (128 rows in each CTA) and B N x 64 (N/2
 // rows in each CTA), issued by the even CTA; each CTA's TMEM receives its 128 rows of D.
 __device__ __forceinline__ void tc_mma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -464,20 +417,6 @@ __device__ __forceinline__ void tc_cp_sf_wide_pair(uint32_t taddr, uint64_t sdes
 
 __device__ __forceinline__ void tc_cp_sf_wide(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// mbarrier wait with cluster-scope acquire: for barriers that other CTAs of the cluster arrive on
-// after writing shared memory the waiter then reads (through tcgen05).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 
 }  // namespace macaq
