@@ -155,7 +155,7 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
  *   mode == MACAQ_A_BF16_FUSED: A = X device bf16 [M, K], inv_s device fp32 [K] (NULL = 1), had_block
  *                               b in {1, 16, 32, 64, 128}; Asf is ignored. The call quantizes X
  *                               bit-identically to macaq_act_quant, so Y equals macaq_act_quant
- *                               followed by the quantized mode. M <= 16 with K % 256 == 0: inside the
+ *                               followed by the quantized mode. M <= 4 with K % 256 == 0: inside the
  *                               skinny kernel (quantizer warps write the MMA's operand stages; no
  *                               quantized activation in HBM). Otherwise: a quantizer pass into the
  *                               workspace, then the GEMM, in stream order. Needs a workspace of

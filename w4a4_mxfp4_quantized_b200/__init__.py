@@ -202,7 +202,7 @@ def linear(A: torch.Tensor, Asf: torch.Tensor | None, Wq: torch.Tensor, Wsf: tor
     kernel (weights in the MMA's M slot, split over all SMs); use_workspace=False runs the general
     kernel instead.
     mode=A_BF16_FUSED: A is bf16 X [M, K]; the call applies inv_s, H_b and MXFP4 itself (inside the
-    GEMM kernel for M <= 16) and needs a workspace."""
+    GEMM kernel for M <= 4) and needs a workspace."""
     N = Wq.shape[0]
     K = Wq.shape[1] * 2
     M = A.shape[0]

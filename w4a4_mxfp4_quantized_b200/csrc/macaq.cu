@@ -577,7 +577,7 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
     return f;
 }
 
-// Y = (X diag(1/s) H_b, MXFP4) x W'^T from bf16 X. Dense calls with M <= 16 and K % 256 == 0 run the
+// Y = (X diag(1/s) H_b, MXFP4) x W'^T from bf16 X. Dense calls with M <= 4 and K % 256 == 0 run the
 // skinny kernel with its quantizer warps: no quantized activation touches HBM. Every other shape (and
 // every grouped call) quantizes X into the workspace and runs the GEMM on it, two launches in stream
 // order: re-quantizing an A tile for every output tile it meets would cost more than the
