@@ -86,6 +86,26 @@ def test_prep_and_linear_reject_bad_shapes(lib):
     assert lib.macaq_grouped_linear(0, P, P, None, P, 0, 16, 256, 256, 32, P, P, P, 0, None, 0, None) == 2
 
 
+def test_fused_mode_rejects_bad_arguments(lib):
+    # mode 1 = MACAQ_A_BF16_FUSED: bf16 X in, inv_s, had_block; checked before any CUDA call
+    args = lambda **kw: [kw.get(k, d) for k, d in (
+        ("mode", 1), ("A", P), ("Asf", None), ("inv", P), ("M", 16), ("N", 256), ("K", 256), ("b", 32), ("Wq", P),
+        ("Wsf", P), ("Y", P), ("out", 0), ("ws", P), ("wsb", 1 << 20), ("st", None))]
+    assert lib.macaq_linear(*args(b=3)) == 4           # Hadamard block outside {1, 16, 32, 64, 128}
+    assert lib.macaq_linear(*args(K=200)) == 2         # K % 128
+    assert lib.macaq_linear(*args(out=7)) == 1         # out dtype
+    assert lib.macaq_linear(*args(A=None)) == 1        # NULL X
+    assert lib.macaq_linear(*args(A=P + 4)) == 3       # misaligned X
+    assert lib.macaq_linear(*args(ws=P + 8)) == 3      # misaligned workspace
+    assert lib.macaq_linear(*args(M=0)) == 0           # M == 0: no-op
+    assert lib.macaq_linear_fixed_scratch(1, P, None, P, 16, 256, 256, 32, P, P, P, 0, None) == 4
+    g = lambda off, E: lib.macaq_grouped_linear(1, P, None, P, off, E, 16, 256, 256, 32, P, P, P, 0, P, 1 << 20, None)
+    assert g(None, 4) == 1                             # grouped needs offsets
+    assert g(P, 0) == 2                                # E < 1
+    assert mq.fused_workspace_bytes(-1, 256, 256) == 0
+    assert mq.fused_workspace_bytes(16, 200, 256) == 0
+
+
 def test_binding_requires_built_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(mq, "_lib", None)
