@@ -130,6 +130,16 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+METRIC = "W4A4 layer TFLOPS (act_quant + block-scaled GEMM)"
+
+
+def layer_config(M: int, world: int) -> dict:
+    """The workload both arms report on."""
+    return {"workload": f"llama3_8b_up_gate K={K_DIM} N={N_DIM} M={M} b={HAD_BLOCK}", "M": M, "N": N_DIM,
+            "K": K_DIM, "had_block": HAD_BLOCK, "parallelism": f"replicas x{world}",
+            "l2": f"inputs rotate over {copies_for(M)} copies (> 2x L2)"}
+
+
 # ------------------------------------------------------------------------------------ ranks
 def max_over_ranks(ms: float, dist_on: bool, device) -> float:
     """The slowest rank's time: every rank runs its own replica, the job ends with the last one."""
@@ -411,11 +421,11 @@ def main():
             cb = cpu_baseline(args.M, budget_s=max(2.0, 60.0 / steps))
             vals.append(cb["value"])
         v = statistics.mean(vals)
-        out = {"impl": "reference", "metric": "W4A4 layer TFLOPS", "value": v, "unit": "TFLOPS",
+        out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS",
                "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
                "ms_per_step": 2.0 * args.M * N_DIM * K_DIM / (v * 1e12) * 1e3, "higher_is_better": True,
                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "config": {"workload": f"llama3_8b_up_gate K={K_DIM} N={N_DIM} M={args.M} b={HAD_BLOCK}"},
+               "config": layer_config(args.M, args.gpus),
                "cpu_baseline": dict(cb, value=v),
                "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(out))
@@ -482,13 +492,11 @@ def main():
             torch.distributed.destroy_process_group()
         return
     out = {
-        "metric": "W4A4 layer TFLOPS (act_quant + block-scaled GEMM)",
+        "metric": METRIC,
         "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "mxfp4 (e2m1 x e2m1, e8m0 scales, fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": f"llama3_8b_up_gate K={K_DIM} N={N_DIM} M={M} b={HAD_BLOCK}", "M": M, "N": N_DIM,
-                   "K": K_DIM, "had_block": HAD_BLOCK, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs rotate over {copies_for(M)} copies (> 2x L2)"},
+        "config": layer_config(M, world),
         "roofline": {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops,
                      "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
                      "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16} (nominal FP4/BF16)",
