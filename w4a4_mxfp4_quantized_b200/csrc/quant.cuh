@@ -152,9 +152,9 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&raw)[4], uint64_t (
 }
 
 // Work split: the K axis is cut into column slabs of slab_groups groups; a tile is tile_rows rows of
-// one slab (always 256 groups, 16 KB). A CTA keeps one slab for its whole life and walks its row
-// tiles, so each consumer thread owns one fixed group column and keeps that column's 32 multipliers
-// in registers. A producer warp streams the tiles with TMA (3-D tensor map rows x 128-byte chunks x
+// one slab (always 256 groups, 16 KB). A CTA keeps one slab for its whole life and walks a
+// contiguous run of its row tiles, so each consumer thread owns one fixed group column and keeps that
+// column's 32 multipliers in registers (reloaded only where the expert changes). A producer warp streams the tiles with TMA (3-D tensor map rows x 128-byte chunks x
 // 64 elements, 128-byte swizzle) into a 4-stage ring with full/empty mbarriers.
 template <int kB, bool kWeight>
 __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a) {
@@ -170,7 +170,11 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
     const int lane = tid & 31;
     const uint32_t slab = blockIdx.x % a.slabs;
     const uint32_t ctas_per_slab = gridDim.x / a.slabs;
-    const uint32_t first_tile = blockIdx.x / a.slabs;
+    // each CTA takes a contiguous run of its slab's row tiles, so the expert (and with it the
+    // per-channel multipliers a thread keeps in registers) changes only at expert boundaries
+    const uint32_t c_in_slab = blockIdx.x / a.slabs;
+    const uint32_t rt_begin = static_cast<uint32_t>(static_cast<uint64_t>(a.row_tiles) * c_in_slab / ctas_per_slab);
+    const uint32_t rt_end = static_cast<uint32_t>(static_cast<uint64_t>(a.row_tiles) * (c_in_slab + 1) / ctas_per_slab);
 
     if (tid == 0) {
         for (int s = 0; s < kQStages; ++s) {
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
             mbar_init(&empty_bar[s], kQConsumerWarps);
         }
         fence_mbar_init();
-        if (first_tile < a.row_tiles) prefetch_tensor_map(&xmap);
+        if (rt_begin < rt_end) prefetch_tensor_map(&xmap);
     }
     griddep_wait();  // X, the offsets and the outputs may belong to the previous kernel in the stream
     load_group_layout(a.offsets, a.E, a.rows, s_off, s_tb);  // contains __syncthreads
@@ -188,7 +192,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
             uint32_t j = 0;
-            for (uint32_t rt = first_tile; rt < a.row_tiles; rt += ctas_per_slab, ++j) {
+            for (uint32_t rt = rt_begin; rt < rt_end; ++rt, ++j) {
                 const int s = j % kQStages;
                 if (j >= kQStages && !mbar_wait(&empty_bar[s], ((j / kQStages) & 1) ^ 1, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&full_bar[s], kQTileBytes);
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
         uint64_t mv[16];
         int cur_e = -1;
         uint32_t j = 0;
-        for (uint32_t rt = first_tile; rt < a.row_tiles; rt += ctas_per_slab, ++j) {
+        for (uint32_t rt = rt_begin; rt < rt_end; ++rt, ++j) {
             const int s = j % kQStages;
             const uint32_t m = rt * a.tile_rows + r_in;
             const bool valid = m < a.rows;
