@@ -190,8 +190,9 @@ macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const
  *   - Sizes whose skinny plan needs more than MACAQ_FIXED_SCRATCH_BYTES (what
  *     macaq_workspace_bytes(M, N, K, 0) reports) are rejected with MACAQ_ERR_WORKSPACE before
  *     anything is launched.
- *   - Only the per-tile counters must start at zero; each call clears them on `stream` (a memset of
- *     at most a few KB) before its kernel, so a call after a MACAQ_ERR_TIMEOUT needs no clean-up.
+ *   - Only the per-tile counters must start at zero; each call clears the ones it uses on `stream`
+ *     (a memset of 4 bytes per 128-row weight tile, rounded up to 256 bytes) before its kernel, so
+ *     a call after a MACAQ_ERR_TIMEOUT needs no clean-up.
  *   - All calls on one device share the one scratch area: two calls whose kernels may overlap
  *     (different streams, or different host threads without ordering) race and give wrong results.
  *     Order them on one stream, or use macaq_linear with separate workspaces.
