@@ -39,6 +39,16 @@ def test_library_exports_every_declared_symbol(lib):
         assert f.read(4) == b"\x7fELF"
 
 
+def test_constants_match_the_header():
+    """The binding and the tests restate two sizes the header defines: keep them in step."""
+    text = open(HEADER).read()
+    counters = re.search(r"#define MACAQ_WORKSPACE_COUNTER_BYTES \(\(size_t\)(\d+)\)", text)
+    fixed = re.search(r"#define MACAQ_FIXED_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert counters and int(counters.group(1)) == mq.WORKSPACE_COUNTER_BYTES
+    import test_zz_no_alloc
+    assert fixed and int(fixed.group(1)) << int(fixed.group(2)) == test_zz_no_alloc.FIXED_SCRATCH_BYTES
+
+
 def test_size_helpers(lib):
     assert mq.sf_bytes(1, 128) == 128 * 4
     assert mq.sf_bytes(128, 4096) == 128 * 128
