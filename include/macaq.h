@@ -136,7 +136,9 @@ macaq_status macaq_prep_weights(const void *W, const float *s, int64_t N, int64_
  *                  non-decreasing, offsets[0] = 0,
  *                  offsets[E] = M: rows [offsets[e], offsets[e+1]) belong to expert e and use
  *                  inv_s + e*K. The values are read on the device; out-of-range offsets are clamped
- *                  into [0, M] so no access leaves the buffers, but give undefined results.
+ *                  into [0, M] so no access leaves the buffers, but give undefined results. A caller
+ *                  that holds a host copy can reject such offsets first with
+ *                  macaq_check_group_offsets().
  *   Xq             device u8 [M, K/2] (written)
  *   Xsf            device u8 (written): dense: macaq_sf_bytes(M, K) bytes; grouped: the per-expert
  *                  padded tiling, at most macaq_grouped_sf_bytes(M, E, K) bytes. Padding rows get 0.
@@ -185,14 +187,16 @@ macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const
  * with M <= 128 and K % 256 == 0 run the skinny kernel on a scratch area that lives in the
  * library's static device data (MACAQ_FIXED_SCRATCH_BYTES per device); every other shape runs the
  * general kernels, which need no scratch.
- *   - The first call on each device looks the scratch's address up (with that device current) and
- *     may load the module; make that first call before any stream capture.
+ *   - Every call looks the scratch's device address up on the current device (a host-side table
+ *     lookup once the module is loaded; nothing is cached, so a device reset does no harm). The
+ *     first call on a device may load the module: make that first call before any stream capture.
  *   - Sizes whose skinny plan needs more than MACAQ_FIXED_SCRATCH_BYTES (what
  *     macaq_workspace_bytes(M, N, K, 0) reports) are rejected with MACAQ_ERR_WORKSPACE before
  *     anything is launched.
  *   - Only the per-tile counters must start at zero; each call clears the ones it uses on `stream`
- *     (a memset of 4 bytes per 128-row weight tile, rounded up to 256 bytes) before its kernel, so
- *     a call after a MACAQ_ERR_TIMEOUT needs no clean-up.
+ *     (a memset of 4 bytes per 128-row weight tile, rounded up to 256 bytes) right before its kernel,
+ *     after every argument check, so a refused call enqueues nothing and a call after a
+ *     MACAQ_ERR_TIMEOUT needs no clean-up.
  *   - All calls on one device share the one scratch area: two calls whose kernels may overlap
  *     (different streams, or different host threads without ordering) race and give wrong results.
  *     Order them on one stream, or use macaq_linear with separate workspaces.
@@ -221,6 +225,15 @@ macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *As
                                   int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf,
                                   void *Y, int32_t out_dtype, void *workspace, size_t ws_bytes,
                                   macaq_stream_t stream);
+
+/*
+ * Host-side check of grouped row offsets (no CUDA call): host_offsets[0..E] must start at 0, end at
+ * total_rows and never decrease, with 1 <= E <= 16384. Returns MACAQ_OK, MACAQ_ERR_SHAPE for offsets
+ * that break a rule, or MACAQ_ERR_INVALID_ARG for a NULL pointer. The device-side reads of the same
+ * offsets (macaq_act_quant, macaq_grouped_linear) clamp instead of failing, because a kernel cannot
+ * return an error before it has read them.
+ */
+macaq_status macaq_check_group_offsets(const int32_t *host_offsets, int32_t E, int64_t total_rows);
 
 /*
  * Reads the sticky device status word that bounded device waits set when they run out. Call it

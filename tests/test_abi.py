@@ -122,3 +122,23 @@ def test_binding_requires_built_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mq, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         mq.lib()
+
+
+def test_host_offsets_check(lib):
+    """Grouped offsets that the device would clamp are rejected on the host (no GPU needed)."""
+    import numpy as np
+
+    mq.check_group_offsets([0, 5, 5, 140, 300], 300)                  # valid, with an empty expert
+    mq.check_group_offsets(np.array([0, 0], np.int32), 0)             # one empty expert, no rows
+    for bad, rows in [([1, 5, 300], 300),                              # does not start at 0
+                      ([0, 5, 299], 300),                              # does not end at total_rows
+                      ([0, 7, 5, 300], 300),                           # decreasing
+                      ([0, -3, 300], 300),                             # negative
+                      ([0, 400, 300], 300)]:                           # past the end, then back
+        with pytest.raises(mq.MacaqError, match="MACAQ_ERR_SHAPE"):
+            mq.check_group_offsets(bad, rows)
+    with pytest.raises(mq.MacaqError, match="MACAQ_ERR_SHAPE"):
+        mq.check_group_offsets([0], 0)                                 # E = 0
+    assert lib.macaq_check_group_offsets(None, 4, 10) == 1
+    big = np.zeros(16386, np.int32)
+    assert lib.macaq_check_group_offsets(big.ctypes.data, 16385, 0) == 2   # E above 16384

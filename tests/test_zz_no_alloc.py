@@ -86,3 +86,31 @@ def test_fixed_scratch_rejects_plans_beyond_its_size():
     torch.cuda.synchronize()
     assert mq.status_str(status) == "MACAQ_ERR_WORKSPACE"
     assert bool((Y == 3.0).all()), "a refused call must not write Y"
+
+
+def test_fixed_scratch_after_a_timeout_needs_no_clean_up():
+    """A split-tile call whose pipeline waits run out (1 ns limit) reports MACAQ_ERR_TIMEOUT and may
+    leave per-tile counters behind in the fixed scratch; the next call clears the counters it uses,
+    so it matches macaq_linear again without any clean-up by the caller."""
+    M, N, K = 16, 4096, 4096
+    Aq, Asf, Wq, Wsf = operands(77, M, N, K)
+    dA, dW = torch.from_numpy(Aq).cuda(), torch.from_numpy(Wq).cuda()
+    dAsf, dWsf = torch.from_numpy(swizzle(Asf, K)).cuda(), torch.from_numpy(swizzle(Wsf, K)).cuda()
+    ref = mq.linear(dA, dAsf, dW, dWsf, out_dtype=mq.OUT_F32)
+    torch.cuda.synchronize()
+    mq.device_status(reset=True)
+    y32 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    try:
+        mq.set_wait_limit_ns(1)
+        assert fixed_scratch_call(dA, dAsf, dW, dWsf, y32, M, N, K, mq.OUT_F32) == 0
+        torch.cuda.synchronize()
+    finally:
+        mq.set_wait_limit_ns(0)
+    assert mq.device_status(reset=True) == 6
+    T = (abs_dequant(Aq, Asf).cuda() @ abs_dequant(Wq, Wsf).cuda().T)
+    for _ in range(2):
+        y32.fill_(float("nan"))
+        assert fixed_scratch_call(dA, dAsf, dW, dWsf, y32, M, N, K, mq.OUT_F32) == 0
+        torch.cuda.synchronize()
+        assert mq.device_status() == 0
+        assert bool(((y32.double() - ref.double()).abs() <= RTOL * T + 1e-30).all())

@@ -25,7 +25,7 @@ __all__ = [
     "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "fused_workspace_bytes", "WORKSPACE_COUNTER_BYTES",
     "status_str",
     "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
-    "set_wait_limit_ns",
+    "set_wait_limit_ns", "check_group_offsets",
     "library_path", "lib",
 ]
 
@@ -60,6 +60,7 @@ _SIGNATURES = {
                               _sz, _vp], ctypes.c_int),
     "macaq_device_status": ([ctypes.POINTER(ctypes.c_int32), _i32], ctypes.c_int),
     "macaq_set_wait_limit_ns": ([ctypes.c_uint64], None),
+    "macaq_check_group_offsets": ([_vp, _i32, _i64], ctypes.c_int),
 }
 
 
@@ -268,3 +269,18 @@ def device_status(reset: bool = False) -> int:
 
 def set_wait_limit_ns(ns: int):
     lib().macaq_set_wait_limit_ns(int(ns))
+
+
+def check_group_offsets(offsets, total_rows: int) -> None:
+    """Host-side check of grouped row offsets (a CPU tensor or array of E + 1 int32 values): they must
+    start at 0, end at total_rows and never decrease. Raises MacaqError(MACAQ_ERR_SHAPE) otherwise.
+    The device-side reads clamp malformed offsets instead of failing, so callers that hold a host
+    copy check it here before launching."""
+    import numpy as np
+
+    a = np.ascontiguousarray(np.asarray(offsets.cpu() if isinstance(offsets, torch.Tensor) else offsets,
+                                        dtype=np.int32))
+    if a.ndim != 1 or a.size < 2:
+        raise MacaqError("macaq_check_group_offsets", 2)
+    _check("macaq_check_group_offsets", lib().macaq_check_group_offsets(
+        a.ctypes.data_as(ctypes.c_void_p), a.size - 1, int(total_rows)))

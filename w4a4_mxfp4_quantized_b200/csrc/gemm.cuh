@@ -909,9 +909,11 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
             const int pidx = static_cast<int>(blockIdx.x - c_first);
             u = u_stop;
             const int b = piece & 1;
-            if (!mbar_wait_or_abort(&accum_full[b], (piece >> 1) & 1, limit, &failed)) break;
+            bool ok = mbar_wait_or_abort(&accum_full[b], (piece >> 1) & 1, limit, &failed);
             tc_fence_after();
-            if (failed) break;
+            // the four epilogue warps meet at named barriers below (split tiles): they stop together
+            // or not at all, so a wait that ran out in one warp never leaves the others at a barrier
+            if (!bar_and(1, 128, ok && !failed)) break;
             const int64_t n = static_cast<int64_t>(tile) * 128 + nl;
             const bool staged = npieces == 1 && !g.out_f32;
             if (staged) {  // the previous tile's store (issued by lane 0) has read the staging buffer

@@ -332,12 +332,17 @@ macaq_status launch_skinny(const CUtensorMap &wmap, const CUtensorMap &xmap, con
                   sfwmap, sfxmap, ymap, g);
 }
 
+// clear_counts > 0: zero that many bytes at the start of the workspace on `st` right before the
+// launch, once every argument and descriptor has been accepted (the fixed-scratch entry point).
 macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, int32_t fused_b, int64_t M, int64_t N,
                         int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
-                        size_t ws_bytes, int sms, cudaStream_t st) {
+                        size_t ws_bytes, int sms, cudaStream_t st, size_t clear_counts = 0) {
     const bool fused = fused_b > 0;
     const SkinnyPlan p = skinny_plan(M, N, K, sms, fused);
     if (!p.ok) return MACAQ_ERR_SHAPE;
+    // the in-kernel quantizer warps take the stages in turn, four at a time: a stage count that is
+    // not a multiple of four would give one stage to two warps at different phases
+    if (fused && p.stages % 4 != 0) return MACAQ_ERR_UNSUPPORTED;
     if (ws_bytes < p.partial_bytes + p.count_bytes) return MACAQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MACAQ_ERR_ALIGNMENT;
     CUtensorMap wmap, xmap, sfwmap, sfxmap, ymap;
@@ -385,6 +390,10 @@ macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, i
     g.gran = p.gran;
     g.wait_limit_ns = g_wait_limit_ns.load();
     g.inv_s = inv_s;
+    if (clear_counts > 0) {
+        const cudaError_t e = cudaMemsetAsync(workspace, 0, clear_counts, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
     switch (fused_b) {
         case 0: return launch_skinny<0>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
         case 1: return launch_skinny<1>(wmap, xmap, sfwmap, sfxmap, ymap, g, p, st);
@@ -505,49 +514,44 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
 // ------------------------------------------------------------------------ fixed scratch
 // Scratch of the skinny kernel for callers that may not allocate device memory: it is part of the
 // module's static device data, so it exists as soon as the module is loaded on a device.
-constexpr int kMaxDevices = 64;
 __device__ __align__(256) uint8_t g_fixed_scratch[MACAQ_FIXED_SCRATCH_BYTES];
 
-// Device address of g_fixed_scratch on the current device, looked up once per device.
+// Device address of g_fixed_scratch on the current device. In host code the symbol is only a
+// host-side stand-in, so the address is looked up on every call (a host-side table lookup once the
+// module is loaded); nothing is cached, so a device reset that reloads the module is harmless.
 macaq_status fixed_scratch(void **out) {
-    static std::mutex mu;
-    static std::array<void *, kMaxDevices> addr{};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fixed_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (dev < 0 || dev >= kMaxDevices) return MACAQ_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_fixed_scratch);
-        if (e != cudaSuccess) return cuda_fail(e);
-        addr[dev] = p;
-    }
-    *out = addr[dev];
+    *out = p;
     return MACAQ_OK;
 }
 
 macaq_status linear_fixed_scratch(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K,
                                   const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype,
                                   cudaStream_t st) {
-    void *scratch = nullptr;
-    macaq_status s = fixed_scratch(&scratch);
-    if (s != MACAQ_OK) return s;
     const bool skinny = M >= 1 && M <= kSkinnyMaxM && N > 0 && N % 128 == 0 && K > 0 && K % 256 == 0 &&
                         N < (int64_t(1) << 31) && K < (int64_t(1) << 31);
     if (!skinny) return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, nullptr, 0, st);
-    if (A == nullptr || Asf == nullptr || Wq == nullptr || Wsf == nullptr || Y == nullptr) return MACAQ_ERR_INVALID_ARG;
+    // every check of the skinny path comes before the counter clear, so a refused call enqueues nothing
     if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
+    if (A == nullptr || Asf == nullptr || Wq == nullptr || Wsf == nullptr || Y == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(Asf) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(Y))
+        return MACAQ_ERR_ALIGNMENT;
     DeviceInfo dev;
-    s = device_info(&dev);
+    macaq_status s = device_info(&dev);
     if (s != MACAQ_OK) return s;
     const SkinnyPlan p = skinny_plan(M, N, K, dev.sms);
     if (!p.ok) return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, nullptr, 0, st);
     if (p.partial_bytes + p.count_bytes > MACAQ_FIXED_SCRATCH_BYTES) return MACAQ_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    s = fixed_scratch(&scratch);
+    if (s != MACAQ_OK) return s;
+    // only the per-tile counters this call uses must start at zero; run_skinny clears them on `st`
+    // after its descriptors are built, immediately before the launch
     const size_t used_counts = (static_cast<size_t>(p.tiles) * 4 + 255) / 256 * 256;
-    const cudaError_t e = cudaMemsetAsync(scratch, 0, used_counts, st);  // the per-tile counters this call uses
-    if (e != cudaSuccess) return cuda_fail(e);
-    return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, scratch, MACAQ_FIXED_SCRATCH_BYTES, st);
+    return run_skinny(A, Asf, nullptr, 0, M, N, K, Wq, Wsf, Y, out_dtype, scratch, MACAQ_FIXED_SCRATCH_BYTES, dev.sms,
+                      st, used_counts);
 }
 
 // ------------------------------------------------------------------------ fused layer (a7)
@@ -567,7 +571,8 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
         const SkinnyPlan p = skinny_plan(M, N, K, sms, M <= kSkinnyFusedMaxM);
         if (p.ok) {
             f.gemm_ws = up(p.count_bytes + p.partial_bytes);
-            f.in_kernel = M <= kSkinnyFusedMaxM;
+            // the quantizer warps need a stage count that is a multiple of four (run_skinny checks it)
+            f.in_kernel = M <= kSkinnyFusedMaxM && p.stages % 4 == 0;
         }
     }
     // the activations never overlap the counter region, whichever kernel runs afterwards
@@ -702,6 +707,15 @@ macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *As
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
     return macaq::gemm(static_cast<const uint8_t *>(A), Asf, group_offsets, E, total_rows, N, K, Wq, Wsf, Y,
                        out_dtype, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_check_group_offsets(const int32_t *host_offsets, int32_t E, int64_t total_rows) {
+    if (host_offsets == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (E < 1 || E > 16384 || total_rows < 0) return MACAQ_ERR_SHAPE;
+    if (host_offsets[0] != 0 || static_cast<int64_t>(host_offsets[E]) != total_rows) return MACAQ_ERR_SHAPE;
+    for (int32_t e = 0; e < E; ++e)
+        if (host_offsets[e + 1] < host_offsets[e]) return MACAQ_ERR_SHAPE;
+    return MACAQ_OK;
 }
 
 macaq_status macaq_device_status(int32_t *status_out, int32_t reset) {

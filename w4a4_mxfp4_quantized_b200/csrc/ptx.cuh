@@ -70,6 +70,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
+// Named barrier `id` over `count` threads (whole warps) that also ANDs a predicate across them: every
+// participating thread gets true only if all of them passed true. Lets a group of warps take one
+// decision (e.g. to stop after a wait ran out) so that none is left waiting at a later barrier.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------------------------------------ dependent launch
 // Programmatic dependent launch. griddep_wait: wait until the grids this one depends on (the previous
 // kernel in the stream, when it was launched with the attribute) have completed and their memory is
