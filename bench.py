@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--M", type=int, default=M_MAIN)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--profile", action="store_true", help="eager passes only, for ncu captures")
+    p.add_argument("--details", default=None, help="also write every section's numbers to this JSON file")
     return p.parse_args()
 
 
@@ -279,49 +280,203 @@ def time_graph(fn, steps, stream):
 
 
 def moe_section(dev, hbm, fp4_peak, steps=20):
-    """The grouped path (MoE 30B-A3B gate/up: 128 experts, top-8 of T tokens, Zipf routing) at
-    T = 64, 1024, 8192: grouped act_quant and grouped GEMM, each timed alone by graph replay.
-    The weights (213 MB prepared) exceed L2 by themselves; X rotates over two copies."""
+    """The grouped path (MoE 30B-A3B: 128 experts, top-8 of T tokens, Zipf routing) at T = 64, 1024,
+    8192 for both projections: gate/up (2048 -> 1536) and down (768 -> 2048). Grouped act_quant and
+    grouped GEMM are timed alone by graph replay. The prepared weights (213 MB gate/up, 107 MB down)
+    are read once per call; X rotates over two copies."""
     import w4a4_mxfp4_quantized_b200 as mq
     from w4a4_mxfp4_quantized_b200 import inputs
 
     stream = torch.cuda.current_stream(dev)
-    c0 = inputs.moe_30b_a3b(64, "gate_up")
-    E, N, K = c0.W.shape
-    Wd = c0.W.to(dev)
-    Wq = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
-    Wsf = torch.empty(E, mq.sf_bytes(N, K), dtype=torch.uint8, device=dev)
-    inv = torch.empty(E, K, dtype=torch.float32, device=dev)
-    sd = c0.s.to(dev)
-    for e in range(E):
-        mq.prep_weights(Wd[e], sd[e], HAD_BLOCK, Wq=Wq[e], Wsf=Wsf[e], inv_s=inv[e])
-    del Wd
     out = []
-    for T in (64, 1024, 8192):
-        c = inputs.moe_30b_a3b(T, "gate_up", draw_w=False)
-        off = c.offsets.to(dev)
-        rows = int(c.offsets[-1])
-        counts = (c.offsets[1:] - c.offsets[:-1]).numpy()
-        Xs = [c.X.to(dev), c.X.to(dev).clone()]
-        Xq = [torch.empty(rows, K // 2, dtype=torch.uint8, device=dev) for _ in range(2)]
-        Xsf = [torch.empty(mq.grouped_sf_bytes(rows, E, K), dtype=torch.uint8, device=dev) for _ in range(2)]
-        Y = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
-        aq = time_graph(lambda i: mq.act_quant(Xs[i % 2], inv, HAD_BLOCK, group_offsets=off, Xq=Xq[i % 2],
-                                               Xsf=Xsf[i % 2]), steps, stream)
-        gm = time_graph(lambda i: mq.grouped_linear(Xq[i % 2], Xsf[i % 2], off, Wq, Wsf, Y=Y), steps, stream)
+    for proj in ("gate_up", "down"):
+        c0 = inputs.moe_30b_a3b(64, proj)
+        E, N, K = c0.W.shape
+        Wd = c0.W.to(dev)
+        Wq = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
+        Wsf = torch.empty(E, mq.sf_bytes(N, K), dtype=torch.uint8, device=dev)
+        inv = torch.empty(E, K, dtype=torch.float32, device=dev)
+        sd = c0.s.to(dev)
+        for e in range(E):
+            mq.prep_weights(Wd[e], sd[e], HAD_BLOCK, Wq=Wq[e], Wsf=Wsf[e], inv_s=inv[e])
+        del Wd
+        for T in (64, 1024, 8192):
+            c = inputs.moe_30b_a3b(T, proj, draw_w=False)
+            off = c.offsets.to(dev)
+            rows = int(c.offsets[-1])
+            counts = (c.offsets[1:] - c.offsets[:-1]).numpy()
+            Xs = [c.X.to(dev), c.X.to(dev).clone()]
+            Xq = [torch.empty(rows, K // 2, dtype=torch.uint8, device=dev) for _ in range(2)]
+            Xsf = [torch.empty(mq.grouped_sf_bytes(rows, E, K), dtype=torch.uint8, device=dev) for _ in range(2)]
+            Y = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+            aq = time_graph(lambda i: mq.act_quant(Xs[i % 2], inv, HAD_BLOCK, group_offsets=off, Xq=Xq[i % 2],
+                                                   Xsf=Xsf[i % 2]), steps, stream)
+            gm = time_graph(lambda i: mq.grouped_linear(Xq[i % 2], Xsf[i % 2], off, Wq, Wsf, Y=Y), steps, stream)
+            assert mq.device_status() == 0
+            flops = 2.0 * N * K * rows
+            used = int((counts > 0).sum())
+            g_bytes = used * N * K * 0.53125 + rows * (0.53125 * K + 2 * N)
+            a_bytes = rows * K * (2 + 0.5 + 1 / 32)
+            out.append({"proj": proj, "T": T, "rows": rows, "experts_used": used, "K": K, "N": N,
+                        "grouped_gemm_us": gm * 1e3, "grouped_gemm_tflops": flops / (gm * 1e-3) / 1e12,
+                        "grouped_gemm_gbs": g_bytes / (gm * 1e-3) / 1e9,
+                        "grouped_gemm_frac_fp4_peak": flops / (gm * 1e-3) / 1e12 / fp4_peak,
+                        "grouped_gemm_frac_hbm": g_bytes / (gm * 1e-3) / 1e9 / hbm,
+                        "grouped_act_quant_us": aq * 1e3, "grouped_act_quant_gbs": a_bytes / (aq * 1e-3) / 1e9,
+                        "grouped_act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm})
+            del Xs, Xq, Xsf, Y
+        del Wq, Wsf, inv
+    return {"workload": f"moe_30b_a3b E=128 top-8, gate/up 2048->1536 and down 768->2048, b={HAD_BLOCK}",
+            "points": out}
+
+
+def _rotations(per_copy_bytes):
+    """Input copies so that consecutive steps read HBM, not L2 (the copies exceed twice L2)."""
+    return max(1, int(np.ceil(2 * L2_BYTES / per_copy_bytes)))
+
+
+def prefill_section(dev, hbm, fp4_peak, steps=10):
+    """Large prefill sweep, all eight shapes M in {4096, 16384} x K in {8192, 16384} x N in {8192,
+    28672}: per shape the plain-MXFP4 pipeline (b = 1, no s: act_quant + GEMM), the transform
+    pipeline (1/s, H_32: act_quant + GEMM), the fused call (bf16 X in), and the GEMM and the
+    act_quant alone. Overheads: (B) transform pipeline over the plain pipeline, (A) transform
+    pipeline over the GEMM on pre-quantized A. Inputs are drawn on the GPU with the same recipe."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    stream = torch.cuda.current_stream(dev)
+    out = []
+    for M in inputs.PREFILL_M:
+        for K in inputs.PREFILL_K:
+            for N in inputs.PREFILL_N:
+                c = inputs.large_prefill(M, K, N, device=str(dev))
+                per_copy = N * K * 0.53125 + M * K * (2 + 0.53125) + M * N * 2
+                ncopy = _rotations(per_copy)
+                Wq, Wsf, inv = mq.prep_weights(c.W, c.s, HAD_BLOCK)
+                pWq, pWsf, _ = mq.prep_weights(c.W, None, 1)
+                del c.W
+                L = {"X": [c.X] + [c.X.clone() for _ in range(ncopy - 1)],
+                     "Wq": [Wq] + [Wq.clone() for _ in range(ncopy - 1)],
+                     "Wsf": [Wsf] + [Wsf.clone() for _ in range(ncopy - 1)],
+                     "pWq": [pWq] + [pWq.clone() for _ in range(ncopy - 1)],
+                     "pWsf": [pWsf] + [pWsf.clone() for _ in range(ncopy - 1)],
+                     "Xq": [torch.empty(M, K // 2, dtype=torch.uint8, device=dev) for _ in range(ncopy)],
+                     "Xsf": [torch.empty(mq.sf_bytes(M, K), dtype=torch.uint8, device=dev) for _ in range(ncopy)],
+                     "Y": [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(ncopy)]}
+                ws = torch.zeros(mq.fused_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+                j = lambda i: i % ncopy
+
+                def plain(i):
+                    mq.act_quant(L["X"][j(i)], None, 1, Xq=L["Xq"][j(i)], Xsf=L["Xsf"][j(i)])
+                    mq.linear(L["Xq"][j(i)], L["Xsf"][j(i)], L["pWq"][j(i)], L["pWsf"][j(i)], Y=L["Y"][j(i)])
+
+                def transform(i):
+                    mq.act_quant(L["X"][j(i)], inv, HAD_BLOCK, Xq=L["Xq"][j(i)], Xsf=L["Xsf"][j(i)])
+                    mq.linear(L["Xq"][j(i)], L["Xsf"][j(i)], L["Wq"][j(i)], L["Wsf"][j(i)], Y=L["Y"][j(i)])
+
+                def fused(i):
+                    mq.linear(L["X"][j(i)], None, L["Wq"][j(i)], L["Wsf"][j(i)], mode=mq.A_BF16_FUSED, inv_s=inv,
+                              had_block=HAD_BLOCK, Y=L["Y"][j(i)], workspace=ws)
+
+                def gemm(i):
+                    mq.linear(L["Xq"][j(i)], L["Xsf"][j(i)], L["Wq"][j(i)], L["Wsf"][j(i)], Y=L["Y"][j(i)])
+
+                def aq(i):
+                    mq.act_quant(L["X"][j(i)], inv, HAD_BLOCK, Xq=L["Xq"][j(i)], Xsf=L["Xsf"][j(i)])
+
+                t = {name: time_graph(fn, steps, stream) for name, fn in
+                     (("plain", plain), ("transform", transform), ("fused", fused), ("gemm", gemm), ("act_quant", aq))}
+                assert mq.device_status() == 0
+                flops = 2.0 * M * N * K
+                a_bytes = M * K * (2 + 0.5 + 1 / 32)
+                out.append({"M": M, "K": K, "N": N, "copies": ncopy,
+                            **{f"{k}_ms": v for k, v in t.items()},
+                            "gemm_tflops": flops / (t["gemm"] * 1e-3) / 1e12,
+                            "gemm_frac_fp4_peak": flops / (t["gemm"] * 1e-3) / 1e12 / fp4_peak,
+                            "transform_tflops": flops / (t["transform"] * 1e-3) / 1e12,
+                            "fused_tflops": flops / (t["fused"] * 1e-3) / 1e12,
+                            "act_quant_gbs": a_bytes / (t["act_quant"] * 1e-3) / 1e9,
+                            "act_quant_frac_hbm": a_bytes / (t["act_quant"] * 1e-3) / 1e9 / hbm,
+                            "overhead_B_transform": t["transform"] / t["plain"] - 1.0,
+                            "overhead_B_fused": t["fused"] / t["plain"] - 1.0,
+                            "overhead_A_transform": t["transform"] / t["gemm"] - 1.0,
+                            "overhead_A_fused": t["fused"] / t["gemm"] - 1.0})
+                del L, ws, Wq, Wsf, pWq, pWsf, c
+                torch.cuda.empty_cache()
+    return {"workload": "large prefill, M x K x N in {4096,16384} x {8192,16384} x {8192,28672}, b=32",
+            "points": out}
+
+
+def qwen3_section(dev, hbm, fp4_peak, steps=10):
+    """The Qwen3-32B decoder-layer linears in sequence at M in {1, 8, 64, 4096}: one step = the four
+    act_quants (qkv, o, gate/up and down inputs) and the seven GEMMs (q, k, v, o, gate, up, down);
+    also the same layer with the fused QKV (N = 10240) and GateUp (N = 51200) linears (four GEMMs).
+    The 487.6 M weights (259 MB prepared) exceed L2, so every step reads them from HBM."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    stream = torch.cuda.current_stream(dev)
+    xs0, ws = inputs.qwen3_32b_layer(1, device=str(dev))
+    prepped, keys = {}, {}
+    for name, K, N, key in inputs.QWEN3_32B_LINEARS:
+        prepped[name] = mq.prep_weights(ws[name], xs0[key].s, HAD_BLOCK)
+        keys[name] = key
+    inv = {}
+    for name, _, _, key in inputs.QWEN3_32B_LINEARS:
+        inv.setdefault(key, prepped[name][2])
+    fused_w = {"qkv": mq.prep_weights(torch.cat([ws["q_proj"], ws["k_proj"], ws["v_proj"]]), xs0["qkv"].s, HAD_BLOCK),
+               "gateup": mq.prep_weights(torch.cat([ws["gate_proj"], ws["up_proj"]]), xs0["gateup"].s, HAD_BLOCK)}
+    del ws
+    w_params = sum(K * N for _, K, N, _ in inputs.QWEN3_32B_LINEARS)
+    out = []
+    for M in inputs.QWEN3_32B_M:
+        xs, _ = inputs.qwen3_32b_layer(M, draw_w=False, device=str(dev))
+        A = {key: mq.act_quant(xs[key].X, inv[key], HAD_BLOCK) for key in xs}
+        Y = {name: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for name, _, N, _ in inputs.QWEN3_32B_LINEARS}
+        Yf = {"qkv": torch.empty(M, 10240, dtype=torch.bfloat16, device=dev),
+              "gateup": torch.empty(M, 51200, dtype=torch.bfloat16, device=dev)}
+
+        def layer(i):
+            for key in xs:
+                mq.act_quant(xs[key].X, inv[key], HAD_BLOCK, Xq=A[key][0], Xsf=A[key][1])
+            for name in prepped:
+                mq.linear(A[keys[name]][0], A[keys[name]][1], prepped[name][0], prepped[name][1], Y=Y[name])
+
+        def layer_fused_weights(i):
+            for key in xs:
+                mq.act_quant(xs[key].X, inv[key], HAD_BLOCK, Xq=A[key][0], Xsf=A[key][1])
+            for key in ("qkv", "gateup"):
+                mq.linear(A[key][0], A[key][1], fused_w[key][0], fused_w[key][1], Y=Yf[key])
+            for name in ("o_proj", "down_proj"):
+                mq.linear(A[keys[name]][0], A[keys[name]][1], prepped[name][0], prepped[name][1], Y=Y[name])
+
+        t = time_graph(layer, steps, stream)
+        tf = time_graph(layer_fused_weights, steps, stream)
+        per = {}
+        for name in prepped:
+            per[name] = time_graph(lambda i, n=name: mq.linear(A[keys[n]][0], A[keys[n]][1], prepped[n][0], prepped[n][1],
+                                                                Y=Y[n]), steps, stream) * 1e3
         assert mq.device_status() == 0
-        flops = 2.0 * N * K * rows
-        g_bytes = int((counts > 0).sum()) * N * K * 0.53125 + rows * (0.53125 * K + 2 * N)
-        a_bytes = rows * K * (2 + 0.5 + 1 / 32)
-        out.append({"T": T, "rows": rows, "experts_used": int((counts > 0).sum()),
-                    "grouped_gemm_us": gm * 1e3, "grouped_gemm_tflops": flops / (gm * 1e-3) / 1e12,
-                    "grouped_gemm_gbs": g_bytes / (gm * 1e-3) / 1e9,
-                    "grouped_gemm_frac_fp4_peak": flops / (gm * 1e-3) / 1e12 / fp4_peak,
-                    "grouped_gemm_frac_hbm": g_bytes / (gm * 1e-3) / 1e9 / hbm,
-                    "grouped_act_quant_us": aq * 1e3, "grouped_act_quant_gbs": a_bytes / (aq * 1e-3) / 1e9,
-                    "grouped_act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm})
-        del Xs, Xq, Xsf, Y
-    return {"workload": f"moe_30b_a3b gate/up E={E} top-8 K={K} N={N} b={HAD_BLOCK}", "points": out}
+        flops = 2.0 * M * w_params
+        bytes_ = w_params * 0.53125 + sum(M * xs[k].X.shape[1] * (2 + 2 * 0.53125) for k in xs) + \
+            sum(2 * M * N for _, _, N, _ in inputs.QWEN3_32B_LINEARS)
+        out.append({"M": M, "layer_us": t * 1e3, "layer_tflops": flops / (t * 1e-3) / 1e12,
+                    "layer_frac_fp4_peak": flops / (t * 1e-3) / 1e12 / fp4_peak,
+                    "layer_gbs": bytes_ / (t * 1e-3) / 1e9, "layer_frac_hbm": bytes_ / (t * 1e-3) / 1e9 / hbm,
+                    "layer_fused_qkv_gateup_us": tf * 1e3, "gemm_us": per})
+        del xs, A, Y, Yf
+    return {"workload": "qwen3_32b decoder-layer linears (q,k,v,o,gate,up,down), b=32", "points": out}
+
+
+def copy_ceiling(dev, nbytes, steps=20):
+    """A device-to-device copy that moves nbytes (half read, half written), timed like the kernels:
+    the rate a plain stream of that size reaches on this GPU, for context beside the HBM peak."""
+    n = int(nbytes // 4)
+    ncopy = _rotations(nbytes)
+    src = [torch.empty(n // 2, dtype=torch.int32, device=dev) for _ in range(ncopy)]
+    dst = [torch.empty(n // 2, dtype=torch.int32, device=dev) for _ in range(ncopy)]
+    ms = time_graph(lambda i: dst[i % ncopy].copy_(src[i % ncopy]), steps, torch.cuda.current_stream(dev))
+    return {"bytes": int(nbytes), "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9}
 
 
 def weight_prep_section(dev, hbm, steps=10):
@@ -379,27 +534,106 @@ def time_e2e(M, steps, warmup, dev, L):
     return a.elapsed_time(b) / steps, M * K_DIM * 2, M * N_DIM * 2
 
 
-def cpu_baseline(M, budget_s=12.0):
-    """The oracle as it stands, single-threaded, on a bounded row sample of the same layer."""
+CPU_ROWS = 8  # rows of the layer per oracle worker and sample (fixed, so the per-row rate is reproducible)
+
+
+def cpu_setup(M):
+    """Inputs of the layer for the oracle: X bits, and W' prepared by the oracle (offline, untimed)."""
     import oracle
     from w4a4_mxfp4_quantized_b200 import inputs
 
     c = inputs.llama3_8b_up(M)
-    Wq, Wsf, inv_s = oracle.prep_weights(c.W, c.s, HAD_BLOCK)  # offline, not timed
-    rows, elapsed, done = 1, 0.0, 0
-    while elapsed < budget_s and done < M:
-        n = min(rows, M - done)
-        Xs = c.X[done:done + n]
-        t0 = time.perf_counter()
-        Xq, Xsf = oracle.act_quant(Xs, inv_s, HAD_BLOCK)
-        oracle.linear(Xq, Xsf, Wq, Wsf)
-        elapsed += time.perf_counter() - t0
-        done += n
-        rows *= 2
-    flops = 2.0 * done * N_DIM * K_DIM
-    return {"value": flops / elapsed / 1e12, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
-            "sample": f"{done} of {M} rows of the layer (act_quant + float64 GEMM over all N), "
-                      f"{elapsed:.1f} s single-threaded C"}
+    Wq, Wsf, inv_s = oracle.prep_weights(c.W, c.s, HAD_BLOCK)
+    bits = c.X.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return c, bits, Wq, Wsf, inv_s
+
+
+def cpu_baseline(M, samples=2):
+    """The oracle as it stands, on the host cores: every worker process (one per core) runs
+    act_quant + the float64 GEMM over all N on its own CPU_ROWS rows of the layer; the value is the
+    rows all workers finished / the wall time of the sample (best of `samples`). Also the same work on
+    one core, and the oracle's act_quant and weight prep timed in full on one core (GB/s of
+    2.53125 B per element)."""
+    import oracle
+    from oracle import timing
+
+    c, bits, Wq, Wsf, inv_s = cpu_setup(M)
+    t1 = timing.single_thread_sample(bits[:CPU_ROWS], Wq, Wsf, inv_s, HAD_BLOCK)
+    with timing.LayerPool(Wq, Wsf, inv_s, HAD_BLOCK) as pool:
+        best = None
+        for i in range(samples):
+            wall, rows = pool.sample(bits, CPU_ROWS, start=i * pool.workers * CPU_ROWS)
+            best = wall if best is None else min(best, wall)
+        workers = pool.workers
+    t0 = time.perf_counter()
+    oracle.act_quant(bits, inv_s, HAD_BLOCK)
+    t_aq = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.prep_weights(c.W, c.s, HAD_BLOCK)
+    t_prep = time.perf_counter() - t0
+    per_row = 2.0 * N_DIM * K_DIM
+    return {"value": workers * CPU_ROWS * per_row / best / 1e12, "unit": "TFLOPS", "cores": workers, "kind": "oracle",
+            "sample": f"{workers} processes x {CPU_ROWS} rows of the layer (act_quant + float64 GEMM over all N), "
+                      f"best of {samples}: {best:.2f} s",
+            "single_core_tflops": CPU_ROWS * per_row / t1 / 1e12,
+            "act_quant_gbs_1core": M * K_DIM * 2.53125 / t_aq / 1e9,
+            "weight_prep_gbs_1core": N_DIM * K_DIM * 2.53125 / t_prep / 1e9}
+
+
+def reference_arm(args):
+    """--impl reference: the oracle timed on the host cores on the same workload, metric and unit.
+    One step = one all-core sample (every core's worker on CPU_ROWS rows of the layer)."""
+    from oracle import timing
+
+    _, bits, Wq, Wsf, inv_s = cpu_setup(args.M)
+    walls, rows = [], 0
+    with timing.LayerPool(Wq, Wsf, inv_s, HAD_BLOCK) as pool:
+        for i in range(args.warmup + args.steps):
+            wall, rows = pool.sample(bits, CPU_ROWS, start=i * pool.workers * CPU_ROWS)
+            if i >= args.warmup:
+                walls.append(wall)
+        workers = pool.workers
+    ms = 1e3 * sum(walls) / len(walls)
+    v = rows * 2.0 * N_DIM * K_DIM / (ms * 1e-3) / 1e12
+    sample = f"each step: {workers} processes x {CPU_ROWS} rows of the layer (act_quant + float64 GEMM over all N)"
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": layer_config(args.M, args.gpus),
+            "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": workers, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def _r(x, n=3):
+    return None if x is None else float(f"{x:.{n}g}")
+
+
+def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling):
+    """Short strings of the sections, so that the whole line stays a few KB."""
+    out = {}
+    if sweep:
+        out["sweep"] = " | ".join(
+            f"M{p['M']}: gemm {p['gemm_us']:.1f}us {p['gemm_frac_hbm']:.2f}hbm {p['gemm_frac_fp4_peak']:.2f}fp4, "
+            f"aq {p['act_quant_us']:.1f}us, fused {p['fused_layer_us']:.1f}us" for p in sweep)
+    out["overhead"] = {k: _r(overhead[k]) for k in ("B_vs_plain_mxfp4_pipeline", "A_vs_gemm_on_prequantized_A")}
+    if prefill:
+        out["prefill"] = " | ".join(
+            f"{p['M']}x{p['K']}x{p['N']}: gemm {p['gemm_ms']:.3f}ms {p['gemm_frac_fp4_peak']:.2f}fp4, "
+            f"B {100 * p['overhead_B_transform']:+.1f}%/{100 * p['overhead_B_fused']:+.1f}%, "
+            f"A {100 * p['overhead_A_transform']:+.1f}%, aq {p['act_quant_frac_hbm']:.2f}hbm" for p in prefill["points"])
+    if qwen3:
+        out["qwen3"] = " | ".join(
+            f"M{p['M']}: {p['layer_us']:.0f}us {p['layer_tflops']:.0f}TF {p['layer_frac_hbm']:.2f}hbm "
+            f"{p['layer_frac_fp4_peak']:.2f}fp4, fusedW {p['layer_fused_qkv_gateup_us']:.0f}us" for p in qwen3["points"])
+    if moe:
+        out["moe"] = " | ".join(
+            f"{p['proj']} T{p['T']}: gemm {p['grouped_gemm_us']:.1f}us {p['grouped_gemm_frac_hbm']:.2f}hbm "
+            f"{p['grouped_gemm_frac_fp4_peak']:.2f}fp4, aq {p['grouped_act_quant_frac_hbm']:.2f}hbm" for p in moe["points"])
+    if prep:
+        out["weight_prep"] = f"{prep['us']:.1f}us {prep['frac_hbm']:.2f}hbm"
+    if ceiling:
+        out["copy_ceiling"] = "; ".join(f"{c['bytes'] / 1e6:.1f}MB copy {c['us']:.1f}us {c['gbs']:.0f}GB/s" for c in ceiling)
+    return out
 
 
 def main():
@@ -412,23 +646,8 @@ def main():
     fp4_peak = bf16 * FP4_OVER_BF16
 
     if args.impl == "reference":
-        if rank != 0:
-            return
-        steps = max(1, args.steps)
-        cb = None
-        vals = []
-        for _ in range(steps):
-            cb = cpu_baseline(args.M, budget_s=max(2.0, 60.0 / steps))
-            vals.append(cb["value"])
-        v = statistics.mean(vals)
-        out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS",
-               "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
-               "ms_per_step": 2.0 * args.M * N_DIM * K_DIM / (v * 1e12) * 1e3, "higher_is_better": True,
-               "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "config": layer_config(args.M, args.gpus),
-               "cpu_baseline": dict(cb, value=v),
-               "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(out))
+        if rank == 0:
+            print(json.dumps(reference_arm(args)))
         return
 
     import w4a4_mxfp4_quantized_b200 as mq  # noqa: F401  (fails loudly without the built library)
@@ -459,13 +678,14 @@ def main():
                 "pages_figure_for_context": "2.3% end-to-end, Qwen3-32B in vLLM, hardware not stated"}
     _, _, _, L = time_layer(M, 3, 1, dev, dist_on)
     e2e_ms, h2d, d2h = time_e2e(M, max(3, args.steps // 2), 2, dev, L)
+    del L
     e2e_ms = max_over_ranks(e2e_ms, dist_on, dev)
     e2e_value = job_tflops(world, flops, e2e_ms)
 
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     gemm_kernel = gemm_kernel_name(M)
     aq_bytes = M * K_DIM * (2 + 0.5 + 1 / 32)
-    sweep = []
+    sweep, prefill, qwen3, moe, prep, ceiling = [], None, None, None, None, []
     if not args.no_sweep:
         for m in M_SWEEP:
             tot, aq, gm, Lm = time_layer(m, max(10, args.steps), args.warmup, dev, dist_on, fused=True)
@@ -483,10 +703,13 @@ def main():
                           "act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm,
                           "fused_layer_us": fz * 1e3,
                           "fused_layer_tflops": fl / (fz * 1e-3) / 1e12,
-                          "fused_form": "quantizer warps inside the skinny GEMM" if m <= 16
+                          "fused_form": "quantizer warps inside the skinny GEMM" if m <= 4
                           else "quantizer pass + GEMM in one call"})
-    moe = moe_section(dev, hbm, fp4_peak) if not args.no_sweep else None
-    prep = weight_prep_section(dev, hbm) if not args.no_sweep else None
+        prefill = prefill_section(dev, hbm, fp4_peak)
+        qwen3 = qwen3_section(dev, hbm, fp4_peak)
+        moe = moe_section(dev, hbm, fp4_peak)
+        prep = weight_prep_section(dev, hbm)
+        ceiling = [copy_ceiling(dev, aq_bytes), copy_ceiling(dev, 16384 * 16384 * 2.53125)]
     if rank != 0:
         if dist_on:
             torch.distributed.destroy_process_group()
@@ -509,12 +732,13 @@ def main():
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "clocks": dict(clocks, window="warm replays (1.5 s of this workload) and the timed replay"),
-        "sweep": sweep,
-        "transform_overhead": overhead,
-        "moe": moe,
-        "weight_prep": prep,
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
+    out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling)
+    if args.details:
+        with open(args.details, "w") as f:
+            json.dump({**out, "sweep": sweep, "transform_overhead": overhead, "prefill": prefill, "qwen3": qwen3,
+                       "moe": moe, "weight_prep": prep, "copy_ceiling": ceiling}, f, indent=1)
     print(json.dumps(out))
     if dist_on:
         torch.distributed.destroy_process_group()

@@ -224,3 +224,51 @@ def grouped_linear(Aq, Asf, offsets, Wq, Wsf, rows=None):
     _load().oracle_grouped_linear(_p(Aq, _u8p), _p(Asf, _u8p), _p(off, _i32p), E, _p(r, _i64p), n_rows,
                                   _p(Wq, _u8p), _p(Wsf, _u8p), N, K, _p(Y, _f64p), _p(T, _f64p), _p(work, _f64p))
     return Y, T
+
+
+def _dequant_rows(codes: np.ndarray, sf: np.ndarray, rows=None) -> np.ndarray:
+    """dequant() of the listed rows (all rows when None)."""
+    if rows is None:
+        return dequant(codes, sf)
+    rows = np.asarray(rows, dtype=np.int64)
+    return dequant(codes[rows], sf[rows])
+
+
+def linear_matmul(Aq, Asf, Wq, Wsf, rows=None, n_chunk: int = 4096):
+    """The quantity linear() computes, Y = dq(A) dq(W)^T and T = |dq(A)| |dq(W)|^T in float64, for the
+    listed rows of A, with the sum over k taken by a float64 library matmul instead of the ordered C
+    loop. The dequantization is the same exact C routine (OCP MX v1.0 element and scale values); the
+    sums differ from linear()'s only by float64 rounding, at most about K * 2^-53 of T, far inside the
+    1e-5 * T tolerance the GPU is held to. W is dequantized n_chunk rows at a time."""
+    Aq = np.ascontiguousarray(Aq, dtype=np.uint8)
+    Asf = np.ascontiguousarray(Asf, dtype=np.uint8)
+    a = _dequant_rows(Aq, Asf, rows)
+    a_abs = np.abs(a)
+    N = Wq.shape[0]
+    Y = np.empty((a.shape[0], N), np.float64)
+    T = np.empty((a.shape[0], N), np.float64)
+    for n0 in range(0, N, n_chunk):
+        w = dequant(np.ascontiguousarray(Wq[n0:n0 + n_chunk]), np.ascontiguousarray(Wsf[n0:n0 + n_chunk]))
+        Y[:, n0:n0 + w.shape[0]] = a @ w.T
+        T[:, n0:n0 + w.shape[0]] = a_abs @ np.abs(w).T
+    return Y, T
+
+
+def grouped_linear_matmul(Aq, Asf, offsets, Wq, Wsf, rows=None):
+    """grouped_linear() with the k-sums by a float64 library matmul (see linear_matmul): row m of expert
+    e (offsets[e] <= m < offsets[e+1]) is multiplied by W'_e = Wq[e], Wsf[e] (row-major SF [N, K/32])."""
+    off = np.asarray(offsets, dtype=np.int64)
+    M = int(off[-1])
+    rows = np.arange(M) if rows is None else np.sort(np.asarray(rows, dtype=np.int64))
+    N = Wq.shape[1]
+    Y = np.empty((len(rows), N), np.float64)
+    T = np.empty((len(rows), N), np.float64)
+    expert = np.searchsorted(off, rows, side="right") - 1
+    for e in np.unique(expert):
+        sel = np.nonzero(expert == e)[0]
+        a = _dequant_rows(np.ascontiguousarray(Aq, dtype=np.uint8), np.ascontiguousarray(Asf, dtype=np.uint8),
+                          rows[sel])
+        w = dequant(np.ascontiguousarray(Wq[e]), np.ascontiguousarray(Wsf[e]))
+        Y[sel] = a @ w.T
+        T[sel] = np.abs(a) @ np.abs(w).T
+    return Y, T

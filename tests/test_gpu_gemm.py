@@ -143,10 +143,29 @@ def test_llama3_8b_up_sampled(M):
     y32 = run_linear(gXq, gXsf, gWq, gWsf, M, N, mq.OUT_F32)
     y16 = run_linear(gXq, gXsf, gWq, gWsf, M, N, mq.OUT_BF16)
     assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
-    rng = np.random.default_rng(M)
-    rows = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 6)])) if M > 1 else np.array([0])
-    Y, T = oracle.linear(oXq, oXsf, oWq, oWsf, rows=rows)
+    if M <= 512:
+        rows = np.arange(M)
+    else:  # 256 random rows plus both edge rows of every 128-row tile
+        rng = np.random.default_rng(M)
+        rows = np.unique(np.concatenate([np.arange(0, M, 128), np.arange(127, M, 128),
+                                         rng.choice(M, 256, replace=False)]))
+    Y, T = oracle.linear_matmul(oXq, oXsf, oWq, oWsf, rows=rows)
     assert_close(y32, Y, T, rows)
+
+
+@pytest.mark.parametrize("M,N,K", [(2048, 14336, 4096), (640, 2816, 1536)])
+def test_random_codes_every_output_many_rounds(M, N, K):
+    """Every output of a shape with more tiles than 2-SM pairs (2048 x 14336: 448 tiles of 256 x 256
+    over 74 pairs, 7 persistent rounds; 640 x 2816: 33 tiles with a ragged last row tile), random
+    codes and scales, checked against the float64 oracle over the whole matrix."""
+    Aq, Asf, Wq, Wsf = random_operands(M + N + K, M, N, K)
+    dA, dW = torch.from_numpy(Aq).cuda(), torch.from_numpy(Wq).cuda()
+    dAsf, dWsf = torch.from_numpy(swizzle(Asf, K)).cuda(), torch.from_numpy(swizzle(Wsf, K)).cuda()
+    y32 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_F32)
+    y16 = run_linear(dA, dAsf, dW, dWsf, M, N, mq.OUT_BF16)
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+    Y, T = oracle.linear_matmul(Aq, Asf, Wq, Wsf)
+    assert_close(y32, Y, T)
 
 
 # ------------------------------------------------------------------------------------- grouped

@@ -282,6 +282,52 @@ def test_linear_row_subset_and_grouped_reduce_to_dense():
     np.testing.assert_array_equal(Yd, Yf[[3, 9]])
 
 
+def test_linear_matmul_equals_the_ordered_sum():
+    """The library-matmul form of the GEMM oracle equals the exact rational sum on tiny shapes and
+    the ordered C loop elsewhere, to float64 rounding (K * 2^-52 of T), with extreme scales, row
+    subsets, W chunking across the chunk size and the grouped form with empty experts."""
+    rng = np.random.default_rng(13)
+    M, N, K = 3, 5, 64
+    Aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    Asf = rng.integers(100, 150, (M, K // 32), dtype=np.uint8)
+    Wsf = rng.integers(100, 150, (N, K // 32), dtype=np.uint8)
+    Y, T = oracle.linear_matmul(Aq, Asf, Wq, Wsf)
+
+    def val(q, sf, r, k):
+        c = (q[r, k // 2] >> (4 * (k & 1))) & 15
+        mag = Fraction(GRID[c & 7])
+        return (-mag if c & 8 else mag) * Fraction(2) ** (int(sf[r, k // 32]) - 127)
+
+    for m in range(M):
+        for n in range(N):
+            terms = [val(Aq, Asf, m, k) * val(Wq, Wsf, n, k) for k in range(K)]
+            tabs = sum((abs(t) for t in terms), Fraction(0))
+            assert abs(Fraction(Y[m, n]) - sum(terms, Fraction(0))) <= Fraction(1, 10 ** 12) * tabs
+            assert abs(Fraction(T[m, n]) - tabs) <= Fraction(1, 10 ** 12) * tabs
+    M, N, K = 37, 300, 1024
+    Aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    Asf = rng.integers(1, 254, (M, K // 32), dtype=np.uint8)
+    Wsf = rng.integers(60, 190, (N, K // 32), dtype=np.uint8)
+    rows = [36, 0, 17]
+    Yl, Tl = oracle.linear(Aq, Asf, Wq, Wsf, rows=rows)
+    Ym, Tm = oracle.linear_matmul(Aq, Asf, Wq, Wsf, rows=rows, n_chunk=128)
+    assert np.all(np.abs(Ym - Yl) <= K * 2.0 ** -52 * Tl)
+    assert np.all(np.abs(Tm - Tl) <= K * 2.0 ** -52 * Tl)
+    E = 4
+    off = np.array([0, 9, 9, 30, 37], np.int32)        # expert 1 is empty
+    Wqe = rng.integers(0, 256, (E, 64, K // 2), dtype=np.uint8)
+    Wsfe = rng.integers(110, 140, (E, 64, K // 32), dtype=np.uint8)
+    Yg, Tg = oracle.grouped_linear(Aq, Asf, off, Wqe, Wsfe)
+    Ygm, Tgm = oracle.grouped_linear_matmul(Aq, Asf, off, Wqe, Wsfe)
+    assert np.all(np.abs(Ygm - Yg) <= K * 2.0 ** -52 * Tg)
+    assert np.all(np.abs(Tgm - Tg) <= K * 2.0 ** -52 * Tg)
+    Ys, _ = oracle.grouped_linear_matmul(Aq, Asf, off, Wqe, Wsfe, rows=[30, 2, 29, 9])
+    sub = [2, 9, 29, 30]
+    assert np.all(np.abs(Ys - Yg[sub]) <= K * 2.0 ** -52 * Tg[sub])
+
+
 # ---------------------------------------------------------------- composed pipeline
 def test_prep_and_act_quant_compose_to_transform_then_quantize():
     g = torch.Generator().manual_seed(21)

@@ -11,6 +11,9 @@ Recipe (every workload):
   * outlier channels: a seeded choice without replacement; those X columns are multiplied by the
     workload's factor;
   * X and W are drawn in fp32 and rounded to bf16 (round-to-nearest-even, torch's cast).
+
+device="cuda" draws the same recipe with a CUDA generator (same shapes and distributions, other
+bits): the benchmark uses it for the large workloads; the parity tests always draw on the CPU.
 """
 from __future__ import annotations
 
@@ -22,23 +25,23 @@ import torch
 LN_LO, LN_HI = math.log(0.5), math.log(8.0)
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator("cpu")
+def _gen(seed: int, device: str = "cpu") -> torch.Generator:
+    g = torch.Generator(device)
     g.manual_seed(int(seed))
     return g
 
 
 def log_uniform_scale(g: torch.Generator, K: int) -> torch.Tensor:
-    u = torch.rand(K, generator=g, dtype=torch.float64)
+    u = torch.rand(K, generator=g, dtype=torch.float64, device=g.device)
     return torch.exp(LN_LO + (LN_HI - LN_LO) * u).to(torch.float32)
 
 
 def outlier_channels(g: torch.Generator, K: int, count: int) -> torch.Tensor:
-    return torch.randperm(K, generator=g)[:count].sort().values
+    return torch.randperm(K, generator=g, device=g.device)[:count].sort().values
 
 
 def normal_bf16(g: torch.Generator, shape, std: float) -> torch.Tensor:
-    return (torch.randn(*shape, generator=g, dtype=torch.float32) * std).to(torch.bfloat16)
+    return (torch.randn(*shape, generator=g, dtype=torch.float32, device=g.device) * std).to(torch.bfloat16)
 
 
 @dataclass
@@ -54,23 +57,23 @@ class DenseCase:
 
 def dense_case(seed: int, M: int, K: int, N: int, *, w_std: float = 0.02, n_outliers: int = 0,
                outlier_factor: float = 1.0, heavy_tail: bool = False, had_block: int = 32,
-               name: str = "dense", draw_w: bool = True) -> DenseCase:
+               name: str = "dense", draw_w: bool = True, device: str = "cpu") -> DenseCase:
     """X ~ N(0, 1) (or sigma_k * N(0, 1) with sigma_k = |t_3| per channel when heavy_tail), with the
     outlier channels scaled by outlier_factor; W ~ N(0, w_std); s log-uniform [0.5, 8]."""
-    g = _gen(seed)
+    g = _gen(seed, device)
     s = log_uniform_scale(g, K)
     out = outlier_channels(g, K, n_outliers)
     if heavy_tail:
         # Student-t with 3 degrees of freedom: z / sqrt(chi2_3 / 3)
-        z = torch.randn(K, generator=g, dtype=torch.float64)
-        chi2 = (torch.randn(3, K, generator=g, dtype=torch.float64) ** 2).sum(0)
+        z = torch.randn(K, generator=g, dtype=torch.float64, device=g.device)
+        chi2 = (torch.randn(3, K, generator=g, dtype=torch.float64, device=g.device) ** 2).sum(0)
         sigma = (z / torch.sqrt(chi2 / 3.0)).abs().to(torch.float32)
     else:
-        sigma = torch.ones(K, dtype=torch.float32)
+        sigma = torch.ones(K, dtype=torch.float32, device=g.device)
     if n_outliers:
         sigma = sigma.clone()
         sigma[out] *= outlier_factor
-    X = (torch.randn(M, K, generator=g, dtype=torch.float32) * sigma).to(torch.bfloat16)
+    X = (torch.randn(M, K, generator=g, dtype=torch.float32, device=g.device) * sigma).to(torch.bfloat16)
     W = normal_bf16(g, (N, K), w_std) if draw_w else None
     return DenseCase(name, X, W, s, had_block, out)
 
@@ -105,18 +108,18 @@ QWEN3_32B_LINEARS = (  # (name, K, N, input id): q/k/v share one input, gate/up 
 QWEN3_32B_M = (1, 8, 64, 4096)
 
 
-def qwen3_32b_layer(M: int, sweep: int = 0, draw_w: bool = True):
+def qwen3_32b_layer(M: int, sweep: int = 0, draw_w: bool = True, device: str = "cpu"):
     """Qwen3-32B-shaped decoder-layer linears. Each distinct input (qkv, o, gateup, down) gets its own
     X (heavy-tailed channel magnitudes) and s; W ~ N(0, 0.02). Returns (inputs dict, weights dict)."""
     inputs = {}
     for i, key in enumerate(("qkv", "o", "gateup", "down")):
         K = {"qkv": 5120, "o": 8192, "gateup": 5120, "down": 25600}[key]
         inputs[key] = dense_case(1000 * 3 + 100 * sweep + i, M, K, 1, heavy_tail=True, n_outliers=0,
-                                 draw_w=False, name=f"qwen3_32b_{key}_M{M}")
+                                 draw_w=False, name=f"qwen3_32b_{key}_M{M}", device=device)
     weights = {}
     if draw_w:
         for j, (name, K, N, _) in enumerate(QWEN3_32B_LINEARS):
-            g = _gen(1000 * 3 + 50 + j)
+            g = _gen(1000 * 3 + 50 + j, device)
             weights[name] = normal_bf16(g, (N, K), 0.02)
     return inputs, weights
 
@@ -189,4 +192,4 @@ def large_prefill(M: int, K: int, N: int, draw_w: bool = True, device: str = "cp
     """Large prefill dense sweep: X ~ N(0,1) with 0.5% outlier channels x50, W ~ N(0, 0.015)."""
     idx = PREFILL_M.index(M) * 4 + PREFILL_K.index(K) * 2 + PREFILL_N.index(N)
     return dense_case(1000 * 5 + idx, M, K, N, w_std=0.015, n_outliers=round(0.005 * K), outlier_factor=50.0,
-                      had_block=32, name=f"prefill_M{M}_K{K}_N{N}", draw_w=draw_w)
+                      had_block=32, name=f"prefill_M{M}_K{K}_N{N}", draw_w=draw_w, device=device)
