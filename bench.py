@@ -279,6 +279,29 @@ def time_graph(fn, steps, stream):
     return ms
 
 
+def time_graphs_interleaved(fns: dict, steps, stream, rounds=3):
+    """Device time per call of each fn(i) (one graph of `steps` calls each), the graphs replayed in
+    turn for `rounds` rounds; each keeps its fastest round. Under the power cap the SM clock drifts
+    over seconds, so pipelines that are compared with each other are timed side by side."""
+    graphs = {}
+    for name, fn in fns.items():
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                fn(i)
+        g.replay()
+        graphs[name] = g
+    best = {name: float("inf") for name in fns}
+    for _ in range(rounds):
+        for name, g in graphs.items():
+            best[name] = min(best[name], replay_ms(g, stream) / steps)
+    del graphs
+    return best
+
+
 def moe_section(dev, hbm, fp4_peak, steps=20):
     """The grouped path (MoE 30B-A3B: 128 experts, top-8 of T tokens, Zipf routing) at T = 64, 1024,
     8192 for both projections: gate/up (2048 -> 1536) and down (768 -> 2048). Grouped act_quant and
@@ -384,8 +407,11 @@ def prefill_section(dev, hbm, fp4_peak, steps=10):
                 def aq(i):
                     mq.act_quant(L["X"][j(i)], inv, HAD_BLOCK, Xq=L["Xq"][j(i)], Xsf=L["Xsf"][j(i)])
 
-                t = {name: time_graph(fn, steps, stream) for name, fn in
-                     (("plain", plain), ("transform", transform), ("fused", fused), ("gemm", gemm), ("act_quant", aq))}
+                def aq_plain(i):
+                    mq.act_quant(L["X"][j(i)], None, 1, Xq=L["Xq"][j(i)], Xsf=L["Xsf"][j(i)])
+
+                t = time_graphs_interleaved({"plain": plain, "transform": transform, "fused": fused, "gemm": gemm,
+                                             "act_quant": aq, "act_quant_plain": aq_plain}, steps, stream)
                 assert mq.device_status() == 0
                 flops = 2.0 * M * N * K
                 a_bytes = M * K * (2 + 0.5 + 1 / 32)
@@ -400,7 +426,11 @@ def prefill_section(dev, hbm, fp4_peak, steps=10):
                             "overhead_B_transform": t["transform"] / t["plain"] - 1.0,
                             "overhead_B_fused": t["fused"] / t["plain"] - 1.0,
                             "overhead_A_transform": t["transform"] / t["gemm"] - 1.0,
-                            "overhead_A_fused": t["fused"] / t["gemm"] - 1.0})
+                            "overhead_A_fused": t["fused"] / t["gemm"] - 1.0,
+                            # the transform's own cost: the only kernel that differs between the two
+                            # pipelines is act_quant (the GEMMs differ only in their operand bits, which
+                            # under the power cap moves the clock and with it the whole-pipeline ratio)
+                            "overhead_B_act_quant_only": (t["act_quant"] - t["act_quant_plain"]) / t["plain"]})
                 del L, ws, Wq, Wsf, pWq, pWsf, c
                 torch.cuda.empty_cache()
     return {"workload": "large prefill, M x K x N in {4096,16384} x {8192,16384} x {8192,28672}, b=32",
@@ -426,6 +456,8 @@ def qwen3_section(dev, hbm, fp4_peak, steps=10):
         inv.setdefault(key, prepped[name][2])
     fused_w = {"qkv": mq.prep_weights(torch.cat([ws["q_proj"], ws["k_proj"], ws["v_proj"]]), xs0["qkv"].s, HAD_BLOCK),
                "gateup": mq.prep_weights(torch.cat([ws["gate_proj"], ws["up_proj"]]), xs0["gateup"].s, HAD_BLOCK)}
+    # gate/up interleaved in blocks of 64 rows for the fused SwiGLU epilogue
+    swiglu_w = mq.prep_weights(mq.interleave_gate_up(ws["gate_proj"], ws["up_proj"]), xs0["gateup"].s, HAD_BLOCK)
     del ws
     w_params = sum(K * N for _, K, N, _ in inputs.QWEN3_32B_LINEARS)
     out = []
@@ -450,8 +482,33 @@ def qwen3_section(dev, hbm, fp4_peak, steps=10):
             for name in ("o_proj", "down_proj"):
                 mq.linear(A[keys[name]][0], A[keys[name]][1], prepped[name][0], prepped[name][1], Y=Y[name])
 
+        I = 25600
+        H = (torch.empty(M, I // 2, dtype=torch.uint8, device=dev), torch.empty(mq.sf_bytes(M, I), dtype=torch.uint8, device=dev))
+        GU = torch.empty(M, 2 * I, dtype=torch.float32, device=dev)
+        ws_sw = torch.zeros(max(int(mq.lib().macaq_linear_swiglu_workspace_bytes(M, 2 * I, 5120)),
+                                mq.workspace_bytes(M, 2 * I, 5120), 1), dtype=torch.uint8, device=dev)
+
+        def swiglu_fused(i):
+            mq.linear_swiglu(A["gateup"][0], A["gateup"][1], swiglu_w[0], swiglu_w[1], inv["down"], HAD_BLOCK,
+                             Hq=H[0], Hsf=H[1], workspace=ws_sw)
+
+        def swiglu_two_step(i):
+            mq.linear(A["gateup"][0], A["gateup"][1], swiglu_w[0], swiglu_w[1], out_dtype=mq.OUT_F32, Y=GU, workspace=ws_sw)
+            mq.swiglu_act_quant(GU, inv["down"], HAD_BLOCK, Hq=H[0], Hsf=H[1])
+
+        def layer_swiglu(i):   # q, k, v, o as in layer(); gate/up with the fused epilogue feeding down
+            for key in ("qkv", "o"):
+                mq.act_quant(xs[key].X, inv[key], HAD_BLOCK, Xq=A[key][0], Xsf=A[key][1])
+            mq.act_quant(xs["gateup"].X, inv["gateup"], HAD_BLOCK, Xq=A["gateup"][0], Xsf=A["gateup"][1])
+            for name in ("q_proj", "k_proj", "v_proj", "o_proj"):
+                mq.linear(A[keys[name]][0], A[keys[name]][1], prepped[name][0], prepped[name][1], Y=Y[name])
+            swiglu_fused(i)
+            mq.linear(H[0], H[1], prepped["down_proj"][0], prepped["down_proj"][1], Y=Y["down_proj"])
+
         t = time_graph(layer, steps, stream)
         tf = time_graph(layer_fused_weights, steps, stream)
+        tsw = time_graphs_interleaved({"fused": swiglu_fused, "two_step": swiglu_two_step, "layer": layer_swiglu},
+                                      steps, stream)
         per = {}
         for name in prepped:
             per[name] = time_graph(lambda i, n=name: mq.linear(A[keys[n]][0], A[keys[n]][1], prepped[n][0], prepped[n][1],
@@ -463,8 +520,10 @@ def qwen3_section(dev, hbm, fp4_peak, steps=10):
         out.append({"M": M, "layer_us": t * 1e3, "layer_tflops": flops / (t * 1e-3) / 1e12,
                     "layer_frac_fp4_peak": flops / (t * 1e-3) / 1e12 / fp4_peak,
                     "layer_gbs": bytes_ / (t * 1e-3) / 1e9, "layer_frac_hbm": bytes_ / (t * 1e-3) / 1e9 / hbm,
-                    "layer_fused_qkv_gateup_us": tf * 1e3, "gemm_us": per})
-        del xs, A, Y, Yf
+                    "layer_fused_qkv_gateup_us": tf * 1e3, "gemm_us": per,
+                    "swiglu_fused_us": tsw["fused"] * 1e3, "swiglu_two_step_us": tsw["two_step"] * 1e3,
+                    "layer_swiglu_chain_us": tsw["layer"] * 1e3})
+        del xs, A, Y, Yf, H, GU, ws_sw
     return {"workload": "qwen3_32b decoder-layer linears (q,k,v,o,gate,up,down), b=32", "points": out}
 
 
@@ -619,12 +678,15 @@ def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling):
     if prefill:
         out["prefill"] = " | ".join(
             f"{p['M']}x{p['K']}x{p['N']}: gemm {p['gemm_ms']:.3f}ms {p['gemm_frac_fp4_peak']:.2f}fp4, "
-            f"B {100 * p['overhead_B_transform']:+.1f}%/{100 * p['overhead_B_fused']:+.1f}%, "
+            f"B {100 * p['overhead_B_transform']:+.1f}%/{100 * p['overhead_B_fused']:+.1f}% "
+            f"(aq only {100 * p['overhead_B_act_quant_only']:+.1f}%), "
             f"A {100 * p['overhead_A_transform']:+.1f}%, aq {p['act_quant_frac_hbm']:.2f}hbm" for p in prefill["points"])
     if qwen3:
         out["qwen3"] = " | ".join(
             f"M{p['M']}: {p['layer_us']:.0f}us {p['layer_tflops']:.0f}TF {p['layer_frac_hbm']:.2f}hbm "
-            f"{p['layer_frac_fp4_peak']:.2f}fp4, fusedW {p['layer_fused_qkv_gateup_us']:.0f}us" for p in qwen3["points"])
+            f"{p['layer_frac_fp4_peak']:.2f}fp4, fusedW {p['layer_fused_qkv_gateup_us']:.0f}us, "
+            f"swiglu chain {p['layer_swiglu_chain_us']:.0f}us (gate/up+swiglu {p['swiglu_fused_us']:.0f} vs "
+            f"{p['swiglu_two_step_us']:.0f}us)" for p in qwen3["points"])
     if moe:
         out["moe"] = " | ".join(
             f"{p['proj']} T{p['T']}: gemm {p['grouped_gemm_us']:.1f}us {p['grouped_gemm_frac_hbm']:.2f}hbm "

@@ -150,6 +150,39 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
                              macaq_stream_t stream);
 
 /*
+ * Activation quantization with a row gather, the dispatch step of a mixture-of-experts layer: output
+ * row m is MXFP4( X[row_index[m]] * diag(inv_s) * H_b ), bit-identical to macaq_act_quant applied
+ * to the gathered copy X[row_index], which is never written to memory.
+ *   X              device bf16 [x_rows, K] (read), e.g. the hidden states in token order
+ *   x_rows         rows of X (>= 1 when M > 0)
+ *   row_index      device int32 [M] (16-byte aligned): the X row of every output row, e.g. the token
+ *                  of each routed row sorted by expert. Values outside [0, x_rows) are clamped into
+ *                  it, so no access leaves X; such a row gets the clamped row's result.
+ *   inv_s, M, K, had_block, group_offsets, E, Xq, Xsf: as for macaq_act_quant, over the M output rows.
+ * Sources: as macaq_act_quant; glonce.com page, paragraph 5 (grouped matmul).
+ */
+macaq_status macaq_act_quant_gather(const void *X, int64_t x_rows, const int32_t *row_index, const float *inv_s,
+                                    int64_t M, int64_t K, int32_t had_block, const int32_t *group_offsets, int32_t E,
+                                    uint8_t *Xq, uint8_t *Xsf, macaq_stream_t stream);
+
+/*
+ * Weighted top-k combine after the down projection of a mixture-of-experts layer:
+ *     out[t, n] = sum over j = 0 .. topk-1 of fl32( weights[t, j] * Y[pos[t, j], n] )
+ * accumulated in fp32 in the order j = 0, 1, ... from +0, every product and every sum rounded on its
+ * own (no multiply-add); bf16 output is the round-to-nearest-even cast of that fp32 value.
+ *   Y        device bf16 [y_rows, N] (read): a grouped linear's output, rows in expert-sorted order
+ *   pos      device int32 [T, topk] (4-byte aligned): the Y row of token t's j-th expert choice;
+ *            values outside [0, y_rows) contribute nothing (a dropped choice)
+ *   weights  device fp32 [T, topk] (4-byte aligned): the router weights
+ *   out      device [T, N] (written), bf16 or fp32 per out_dtype
+ *   N % 8 == 0, 1 <= topk <= 1024, T >= 0 (T == 0 is a no-op); Y and out 16-byte aligned.
+ * Source: glonce.com page, paragraph 5 (grouped matmul); the combine returns the grouped GEMM's rows
+ * to token order.
+ */
+macaq_status macaq_moe_combine(const void *Y, int64_t y_rows, int64_t N, const int32_t *pos, const float *weights,
+                               int64_t T, int32_t topk, void *out, int32_t out_dtype, macaq_stream_t stream);
+
+/*
  * Dense W4A4 linear: Y[m, n] = sum_k dq(A[m, k]) * dq(W'[n, k]), fp32 accumulation on the tcgen05
  * tensor cores (kind::mxf4 block-scaled MMA), written as bf16 (round-to-nearest-even) or fp32.
  *   mode == MACAQ_A_QUANTIZED:  A = Xq device u8 [M, K/2], Asf = Xsf (tiled, macaq_sf_bytes(M, K)),
@@ -204,6 +237,45 @@ macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const
 macaq_status macaq_linear_fixed_scratch(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
                                         int64_t M, int64_t N, int64_t K, int32_t had_block, const uint8_t *Wq,
                                         const uint8_t *Wsf, void *Y, int32_t out_dtype, macaq_stream_t stream);
+
+/*
+ * Gate/up linear of a SwiGLU MLP with the down projection's activation quantization fused after it:
+ *     G, U = X' * W'_gu^T            (the block-scaled GEMM, fp32 accumulation)
+ *     H    = silu(G) * U             (fp32; silu(g) = g / (1 + exp(-g)) with one fixed fp32 exp)
+ *     Hq, Hsf = MXFP4( H * diag(inv_s_down) * H_b )    (the macaq_act_quant arithmetic)
+ * so that Hq/Hsf are the A operand of the down projection's macaq_linear. The fixed exp is Cody and
+ * Waite's reduction n = rint(x log2 e), r = (x - n C1) - n C2 (C1 = 0x3F317200, C2 = 0x35BFBE8E as
+ * fp32 bit patterns), the Taylor polynomial sum_{k=0..6} r^k / k! by Horner's rule, times 2^n, x
+ * clamped to [-100, 88], each step one round-to-nearest fp32 operation with no multiply-add.
+ *   A, Asf      the gate/up input, quantized (macaq_act_quant) as for macaq_linear: u8 [M, K/2] + SF
+ *   N           2 * I, a multiple of 256 (I intermediate channels)
+ *   Wq, Wsf     the gate/up weights prepared by macaq_prep_weights from one [N, K] matrix whose rows
+ *               interleave the two projections in blocks of 64: gate rows 64j..64j+63, then up rows
+ *               64j..64j+63, for j = 0 .. I/64 - 1
+ *   inv_s_down  device fp32 [I]: the down projection's 1/s (from its macaq_prep_weights), or NULL
+ *   had_block_down  the down projection's Hadamard block, in {1, 16, 32, 64}
+ *   Hq          device u8 [M, I/2] (written); Hsf device u8, macaq_sf_bytes(M, I) (written, padding 0)
+ *   workspace   M > 128 with K % 256 == 0: unused (the GEMM's epilogue does the rest; G and U never
+ *               reach memory); otherwise at least macaq_linear_swiglu_workspace_bytes(M, N, K) bytes
+ *               (the GEMM writes G, U in fp32 there, then macaq_swiglu_act_quant's kernel runs), under
+ *               the workspace contract of macaq_workspace_bytes.
+ * Sources: aipolix.com page, paragraph 2 (the transform at the input of every linear); glonce.com
+ * page, paragraph 5 (W4A4 dense matmul). The pages do not define the MLP's activation: the fp32
+ * evaluation above is this library's definition.
+ */
+size_t macaq_linear_swiglu_workspace_bytes(int64_t M, int64_t N, int64_t K);
+macaq_status macaq_linear_swiglu(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K,
+                                 const uint8_t *Wq, const uint8_t *Wsf, const float *inv_s_down, int32_t had_block_down,
+                                 uint8_t *Hq, uint8_t *Hsf, void *workspace, size_t ws_bytes, macaq_stream_t stream);
+
+/*
+ * The second half of macaq_linear_swiglu on a gate/up output already in memory:
+ *   GU      device fp32 [M, 2I], columns interleaved in blocks of 64 (gate 64j.., then up 64j..)
+ *   I       a multiple of 128; inv_s [I] or NULL; had_block in {1, 16, 32, 64}
+ *   Hq, Hsf as for macaq_linear_swiglu.
+ */
+macaq_status macaq_swiglu_act_quant(const float *GU, int64_t M, int64_t I, const float *inv_s, int32_t had_block,
+                                    uint8_t *Hq, uint8_t *Hsf, macaq_stream_t stream);
 
 /*
  * Grouped (MoE) W4A4 linear: rows [offsets[e], offsets[e+1]) of A are multiplied by expert e's

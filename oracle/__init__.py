@@ -71,6 +71,14 @@ def _load():
             lib.oracle_linear.argtypes = [_u8p, _u8p, _i64p, _i64, _u8p, _u8p, _i64, _i64, _f64p, _f64p, _f64p]
             lib.oracle_grouped_linear.argtypes = [_u8p, _u8p, _i32p, ctypes.c_int32, _i64p, _i64, _u8p, _u8p,
                                                   _i64, _i64, _f64p, _f64p, _f64p]
+            lib.oracle_bf16_rne.argtypes = [ctypes.c_float]
+            lib.oracle_bf16_rne.restype = ctypes.c_uint16
+            lib.oracle_moe_combine.argtypes = [_u16p, _i64, _i64, _i32p, _f32p, _i64, ctypes.c_int32, _f32p]
+            lib.oracle_exp_f32.argtypes = [ctypes.c_float]
+            lib.oracle_exp_f32.restype = ctypes.c_float
+            lib.oracle_swiglu_f32.argtypes = [ctypes.c_float, ctypes.c_float]
+            lib.oracle_swiglu_f32.restype = ctypes.c_float
+            lib.oracle_swiglu_act_quant.argtypes = [_f32p, _f32p, _f32p, _i64, _i64, ctypes.c_int, _u8p, _u8p, _f32p]
             _lib = lib
     return _lib
 
@@ -272,3 +280,47 @@ def grouped_linear_matmul(Aq, Asf, offsets, Wq, Wsf, rows=None):
         Y[sel] = a @ w.T
         T[sel] = np.abs(a) @ np.abs(w).T
     return Y, T
+
+
+def bf16_rne(values) -> np.ndarray:
+    """fp32 values -> bf16 bit patterns (uint16), round to nearest even."""
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float32)).ravel()
+    lib = _load()
+    return np.array([lib.oracle_bf16_rne(float(x)) for x in v], dtype=np.uint16).reshape(np.shape(values))
+
+
+def moe_combine(Y_bf16, pos, w) -> np.ndarray:
+    """out[t, n] = sum_j fl32(w[t, j] * Y[pos[t, j], n]) in fp32, j in order from +0 (pos outside the
+    rows of Y skipped). Y: bf16 [y_rows, N] (torch CPU tensor or uint16 bits); pos int32 and w fp32
+    [T, topk]. Returns fp32 [T, N]."""
+    y = _bits16(Y_bf16)
+    y_rows, N = y.shape
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int32))
+    w = np.ascontiguousarray(np.asarray(w, dtype=np.float32))
+    T, topk = pos.shape
+    out = np.empty((T, N), np.float32)
+    _load().oracle_moe_combine(_p(y, _u16p), y_rows, N, _p(pos, _i32p), _p(w, _f32p), T, topk, _p(out, _f32p))
+    return out
+
+
+def exp_f32(x: float) -> float:
+    """The fixed fp32 exp of the fused SwiGLU (Cody-Waite reduction, degree-6 Taylor, x in [-100, 88])."""
+    return float(_load().oracle_exp_f32(ctypes.c_float(x)))
+
+
+def swiglu_f32(g: float, u: float) -> float:
+    return float(_load().oracle_swiglu_f32(ctypes.c_float(g), ctypes.c_float(u)))
+
+
+def swiglu_act_quant(G, U, inv_s, b: int):
+    """MXFP4(swiglu(G, U) diag(inv_s) H_b) of fp32 [M, I] gate and up outputs -> (Hq [M, I/2], Hsf [M, I/32])."""
+    G = np.ascontiguousarray(G, dtype=np.float32)
+    U = np.ascontiguousarray(U, dtype=np.float32)
+    M, I = G.shape
+    inv = _f32(inv_s)
+    Hq = np.empty((M, I // 2), np.uint8)
+    Hsf = np.empty((M, I // MX_GROUP), np.uint8)
+    work = np.empty(I, np.float32)
+    _load().oracle_swiglu_act_quant(_p(G, _f32p), _p(U, _f32p), _p(inv, _f32p), M, I, int(b), _p(Hq, _u8p),
+                                    _p(Hsf, _u8p), _p(work, _f32p))
+    return Hq, Hsf

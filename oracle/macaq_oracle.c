@@ -307,3 +307,117 @@ void oracle_grouped_linear(const uint8_t *Aq, const uint8_t *Asf, const int32_t 
         }
     }
 }
+
+/*
+ * fp32 -> bf16 bit pattern, round to nearest, ties to even (finite inputs): the upper 16 bits of the
+ * fp32 pattern after adding 0x7FFF plus the lowest kept bit. This is the cast the GPU path applies
+ * to its fp32 results.
+ */
+uint16_t oracle_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/*
+ * Weighted top-k combine of a mixture-of-experts layer, the plain definition with a fixed order:
+ * out[t, n] = sum over j = 0 .. topk-1 of fl32(w[t, j] * Y[pos[t, j], n]), accumulated in fp32 from
+ * +0 in the order j = 0, 1, ..., every product and sum rounded on its own; choices whose pos is
+ * outside [0, y_rows) are skipped. [MACaQ-en] paragraph 5 (grouped matmul: the combine returns the
+ * expert-sorted rows to token order).
+ *   Y [y_rows, N] bf16 bits, pos/w [T, topk] -> out [T, N] fp32.
+ */
+void oracle_moe_combine(const uint16_t *Y, int64_t y_rows, int64_t N, const int32_t *pos, const float *w,
+                        int64_t T, int32_t topk, float *out)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < topk; ++j) {
+                int64_t p = pos[t * topk + j];
+                if (p < 0 || p >= y_rows)
+                    continue;
+                float prod = w[t * topk + j] * bf16_to_float(Y[p * N + n]);
+                acc = acc + prod;
+            }
+            out[t * N + n] = acc;
+        }
+    }
+}
+
+/*
+ * exp(x) in fp32, the evaluation both sides of the fused SwiGLU use (the pages leave the MLP's
+ * activation function to the model; this fixes one exact fp32 evaluation of it). Method: Cody and
+ * Waite's argument reduction (W. J. Cody, W. Waite, "Software Manual for the Elementary Functions",
+ * 1980): n = rint(x * log2(e)), r = (x - n*C1) - n*C2 with ln 2 = C1 + C2 split so that n*C1 is exact;
+ * then the Taylor polynomial 1 + r + r^2/2! + ... + r^6/6! by Horner's rule, and the result p * 2^n.
+ * Every operation is one fp32 operation rounded to nearest (no multiply-add contraction). x is
+ * clamped to [-100, 88] first, so 2^n is always a representable float (normal or subnormal) and the
+ * final product rounds once.
+ */
+static float f32_from_bits(uint32_t u)
+{
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+float oracle_exp_f32(float x)
+{
+    const float log2e = f32_from_bits(0x3FB8AA3Bu); /* 1.44269504 */
+    const float c1 = f32_from_bits(0x3F317200u);    /* 0.693145751953125 (ln 2, high part) */
+    const float c2 = f32_from_bits(0x35BFBE8Eu);    /* 1.42860677e-06 (ln 2 - c1) */
+    static const float inv_fact[7] = {1.0f, 1.0f, 0.5f, 1.0f / 6.0f, 1.0f / 24.0f, 1.0f / 120.0f, 1.0f / 720.0f};
+    if (x < -100.0f)
+        x = -100.0f;
+    if (x > 88.0f)
+        x = 88.0f;
+    float t = x * log2e;
+    float nf = rintf(t);
+    float a = nf * c1;
+    float r = x - a;
+    float b = nf * c2;
+    r = r - b;
+    float p = inv_fact[6];
+    for (int k = 5; k >= 0; --k) {
+        float pr = p * r;
+        p = pr + inv_fact[k];
+    }
+    int n = (int)nf;                       /* in [-145, 127] */
+    float scale = ldexpf(1.0f, n);         /* 2^n, exact: normal or subnormal */
+    return p * scale;
+}
+
+/* silu(g) * u with silu(g) = g / (1 + exp(-g)), each operation one fp32 rounding. */
+float oracle_swiglu_f32(float g, float u)
+{
+    float e = oracle_exp_f32(-g);
+    float den = 1.0f + e;
+    float s = g / den;
+    return s * u;
+}
+
+/*
+ * The fused gate/up epilogue's output, the plain definition: H[m, i] = swiglu(G[m, i], U[m, i]) in
+ * fp32 (the gate/up GEMM outputs rounded to fp32), then the down projection's activation
+ * quantization of H (its per-channel 1/s and block Hadamard, then MXFP4), exactly as
+ * oracle_act_quant. [MACaQ-fa] paragraph 2 (the transform at the input of every linear, here the
+ * down projection's input).
+ *   G, U [M, I] fp32 -> Hq [M, I/2], Hsf [M, I/32] row-major. work: I floats.
+ */
+void oracle_swiglu_act_quant(const float *G, const float *U, const float *inv_s, int64_t M, int64_t I, int b,
+                             uint8_t *Hq, uint8_t *Hsf, float *work)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t i = 0; i < I; ++i) {
+            float h = oracle_swiglu_f32(G[m * I + i], U[m * I + i]);
+            work[i] = inv_s ? h * inv_s[i] : h;
+        }
+        if (b > 1)
+            for (int64_t k0 = 0; k0 < I; k0 += b)
+                oracle_fwht_f32(work + k0, b);
+        oracle_mxfp4_quantize_row(work, I, Hq + m * (I / 2), Hsf + m * (I / MX_GROUP));
+    }
+}

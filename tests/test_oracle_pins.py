@@ -370,3 +370,96 @@ def test_quantized_layer_approximates_unquantized_product():
         Y, _ = oracle.linear(Xq, Xsf, Wq, Wsf)
         rel = np.linalg.norm(Y - ref) / np.linalg.norm(ref)
         assert rel < bound, rel
+
+
+# ---------------------------------------------------------------- MoE combine
+def test_bf16_rne_matches_torch_cast():
+    """The oracle's fp32 -> bf16 rounding equals torch's round-to-nearest-even cast, including exact
+    ties (odd and even kept bit), subnormals, signed zeros and values near the top of the range."""
+    g = torch.Generator().manual_seed(31)
+    v = torch.randn(4000, generator=g) * torch.exp(torch.randn(4000, generator=g) * 20)
+    ties = torch.tensor([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -130 * 1.5,
+                         1e-40, -0.0, 0.0, 3.0e38, -3.0e38, 2.0 ** -126 * (1 + 2.0 ** -8)])
+    v = torch.cat([v, ties]).to(torch.float32)
+    v = v[torch.isfinite(v)]
+    ref = v.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.bf16_rne(v.numpy()), ref)
+
+
+def test_moe_combine_definition():
+    """Properties that fix the combine: with one choice of weight 1 it copies rows exactly; dropped
+    choices (pos outside Y) equal omitting them; the fp32 result is within the rounding bound of the
+    exact float64 weighted sum (2 * topk roundings of 2^-24 each, relative to sum |w y|)."""
+    g = torch.Generator().manual_seed(32)
+    y_rows, N, T, topk = 40, 24, 9, 6
+    Y = torch.randn(y_rows, N, generator=g).to(torch.bfloat16)
+    pos = torch.randint(0, y_rows, (T, topk), generator=g).to(torch.int32).numpy()
+    w = torch.rand(T, topk, generator=g).numpy().astype(np.float32)
+    one = oracle.moe_combine(Y, pos[:, :1], np.ones((T, 1), np.float32))
+    np.testing.assert_array_equal(one, Y.float().numpy()[pos[:, 0]])
+    out = oracle.moe_combine(Y, pos, w)
+    yd = Y.double().numpy()
+    exact = np.einsum("tj,tjn->tn", w.astype(np.float64), yd[pos])
+    tabs = np.einsum("tj,tjn->tn", np.abs(w.astype(np.float64)), np.abs(yd[pos]))
+    assert np.all(np.abs(out - exact) <= 2 * topk * 2.0 ** -24 * tabs)
+    dropped = pos.copy()
+    dropped[:, 2] = -1
+    dropped[0, 4] = y_rows          # past the end: also skipped
+    got = oracle.moe_combine(Y, dropped, w)
+    keep = [0, 1, 3, 4, 5]           # rows 1.. lose choice 2
+    np.testing.assert_array_equal(got[1:], oracle.moe_combine(Y, pos[1:, keep], w[1:, keep]))
+    keep0 = [0, 1, 3, 5]             # row 0 loses choices 2 and 4
+    np.testing.assert_array_equal(got[:1], oracle.moe_combine(Y, pos[:1, keep0], w[:1, keep0]))
+
+
+# ---------------------------------------------------------------- fused SwiGLU
+def test_exp_f32_against_the_exponential():
+    """The fixed fp32 exp is within 4 ulp of exp over its range, exact at 0, and clamps outside it."""
+    import math
+
+    xs = np.concatenate([np.linspace(-100, 88, 40001), np.float32([-0.0, 1e-30, -1e-30, 0.34657359, -0.34657359,
+                                                                   1.0, -1.0, 87.99, -99.99])]).astype(np.float32)
+    for x in xs:
+        e = oracle.exp_f32(float(x))
+        ref = math.exp(float(x))
+        if ref >= 2.0 ** -126:
+            assert abs(e - ref) <= 4 * float(np.spacing(np.float32(ref))), (x, e, ref)
+        else:   # subnormal results: within 4 units of the smallest subnormal step
+            assert abs(e - ref) <= 4 * 2.0 ** -149, (x, e, ref)
+    assert oracle.exp_f32(0.0) == 1.0
+    assert oracle.exp_f32(-1000.0) == oracle.exp_f32(-100.0)
+    assert oracle.exp_f32(1000.0) == oracle.exp_f32(88.0)
+
+
+def test_swiglu_f32_definition():
+    import math
+
+    rng = np.random.default_rng(41)
+    for g, u in zip(rng.normal(0, 4, 3000).astype(np.float32), rng.normal(0, 2, 3000).astype(np.float32)):
+        ref = float(g) * float(u) / (1.0 + math.exp(-float(g)))
+        got = oracle.swiglu_f32(float(g), float(u))
+        assert abs(got - ref) <= 8 * float(np.spacing(np.float32(abs(ref)))) + 1e-38, (g, u, got, ref)
+    assert oracle.swiglu_f32(0.0, 5.0) == 0.0
+    assert oracle.swiglu_f32(200.0, 3.0) == 600.0          # exp(-200) clamps to exp(-100): silu(g) = g
+    tiny = oracle.swiglu_f32(-200.0, 3.0)                   # exp(200) clamps to exp(88): -200 / (1 + e^88) * 3
+    assert -1e-33 < tiny < 0.0
+
+
+def test_swiglu_act_quant_composes_swiglu_transform_and_mxfp4():
+    """swiglu_act_quant equals: the elementwise fixed SwiGLU, the fp32 multiply by 1/s, the fixed-order
+    butterflies per block, then MXFP4 (each step its own pinned oracle function)."""
+    rng = np.random.default_rng(42)
+    M, I = 5, 256
+    G = rng.normal(0, 3, (M, I)).astype(np.float32)
+    U = rng.normal(0, 1, (M, I)).astype(np.float32)
+    inv = np.exp(rng.uniform(-2.0, 0.7, I)).astype(np.float32)
+    for b in (1, 16, 32, 64):
+        H = np.array([[oracle.swiglu_f32(float(G[m, i]), float(U[m, i])) for i in range(I)] for m in range(M)],
+                     np.float32)
+        V = (H * inv).astype(np.float32)
+        if b > 1:
+            V = np.stack([np.concatenate([oracle.fwht_f32(V[m, k:k + b]) for k in range(0, I, b)]) for m in range(M)])
+        c_ref, s_ref = oracle.mxfp4_quantize(V)
+        c, s = oracle.swiglu_act_quant(G, U, inv, b)
+        np.testing.assert_array_equal(c, c_ref)
+        np.testing.assert_array_equal(s, s_ref)

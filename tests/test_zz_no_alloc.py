@@ -73,10 +73,17 @@ def test_fixed_scratch_matches_linear(M, N, K):
 
 def test_fixed_scratch_rejects_plans_beyond_its_size():
     """A skinny plan that needs more scratch than the fixed area is refused before any launch."""
-    M, N, K = 128, 1024, 65536
-    while mq.workspace_bytes(M, N, K) <= FIXED_SCRATCH_BYTES:
-        K *= 2
-        assert K <= 1 << 20, "no shape found whose skinny plan exceeds the fixed scratch"
+    M = 128
+    shape = None
+    for N in (1024, 4096, 8192, 16384):           # partial tiles grow with tiles x pieces x M
+        for K in (16384, 32768, 65536, 131072):
+            if mq.workspace_bytes(M, N, K) > FIXED_SCRATCH_BYTES:
+                shape = (N, K)
+                break
+        if shape:
+            break
+    assert shape is not None, "no shape found whose skinny plan exceeds the fixed scratch"
+    N, K = shape
     dA = torch.zeros(M, K // 2, dtype=torch.uint8, device="cuda")
     dAsf = torch.zeros(mq.sf_bytes(M, K), dtype=torch.uint8, device="cuda")
     dW = torch.zeros(N, K // 2, dtype=torch.uint8, device="cuda")

@@ -25,7 +25,8 @@ __all__ = [
     "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "fused_workspace_bytes", "WORKSPACE_COUNTER_BYTES",
     "status_str",
     "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
-    "set_wait_limit_ns", "check_group_offsets",
+    "set_wait_limit_ns", "check_group_offsets", "act_quant_gather", "moe_combine",
+    "linear_swiglu", "swiglu_act_quant", "interleave_gate_up",
     "library_path", "lib",
 ]
 
@@ -61,6 +62,11 @@ _SIGNATURES = {
     "macaq_device_status": ([ctypes.POINTER(ctypes.c_int32), _i32], ctypes.c_int),
     "macaq_set_wait_limit_ns": ([ctypes.c_uint64], None),
     "macaq_check_group_offsets": ([_vp, _i32, _i64], ctypes.c_int),
+    "macaq_act_quant_gather": ([_vp, _i64, _vp, _vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
+    "macaq_moe_combine": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _i32, _vp], ctypes.c_int),
+    "macaq_linear_swiglu_workspace_bytes": ([_i64, _i64, _i64], _sz),
+    "macaq_linear_swiglu": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "macaq_swiglu_act_quant": ([_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
 }
 
 
@@ -186,6 +192,80 @@ def act_quant(X: torch.Tensor, inv_s: torch.Tensor | None, had_block: int = 32, 
     _check("macaq_act_quant", lib().macaq_act_quant(
         _ptr(X), _ptr(inv_s), M, K, had_block, _ptr(group_offsets), E, _ptr(Xq), _ptr(Xsf), _stream(dev)))
     return Xq, Xsf
+
+
+def act_quant_gather(X: torch.Tensor, row_index: torch.Tensor, inv_s: torch.Tensor | None, had_block: int = 32, *,
+                     group_offsets=None, Xq=None, Xsf=None):
+    """act_quant of the gathered rows X[row_index] without writing that copy: row m of the output is
+    the transform and MXFP4 of X[row_index[m]] (row_index int32 CUDA [M]). Grouped form as act_quant."""
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and row_index.dtype == torch.int32
+    x_rows, K = X.shape
+    M = row_index.numel()
+    dev = X.device
+    E = 0 if group_offsets is None else group_offsets.numel() - 1
+    Xq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev) if Xq is None else Xq
+    if Xsf is None:
+        n = grouped_sf_bytes(M, E, K) if group_offsets is not None else sf_bytes(M, K)
+        Xsf = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    _check("macaq_act_quant_gather", lib().macaq_act_quant_gather(
+        _ptr(X), x_rows, _ptr(row_index), _ptr(inv_s), M, K, had_block, _ptr(group_offsets), E, _ptr(Xq), _ptr(Xsf),
+        _stream(dev)))
+    return Xq, Xsf
+
+
+def moe_combine(Y: torch.Tensor, pos: torch.Tensor, weights: torch.Tensor, *, out_dtype: int = OUT_BF16, out=None):
+    """out[t] = sum_j weights[t, j] * Y[pos[t, j]] in fp32, j in order (pos outside Y's rows skipped).
+    Y bf16 CUDA [rows, N] (N % 8 == 0); pos int32 and weights fp32 CUDA [T, topk]."""
+    assert Y.dtype == torch.bfloat16 and pos.dtype == torch.int32 and weights.dtype == torch.float32
+    y_rows, N = Y.shape
+    T, topk = pos.shape
+    dev = Y.device
+    out = _out(T, N, out_dtype, dev, out)
+    _check("macaq_moe_combine", lib().macaq_moe_combine(
+        _ptr(Y), y_rows, N, _ptr(pos), _ptr(weights), T, topk, _ptr(out), out_dtype, _stream(dev)))
+    return out
+
+
+def interleave_gate_up(W_gate: torch.Tensor, W_up: torch.Tensor, block: int = 64) -> torch.Tensor:
+    """Stacks gate and up weights [I, K] into the [2I, K] layout linear_swiglu expects: gate rows
+    64j..64j+63, then up rows 64j..64j+63, for every j (pure indexing)."""
+    I, K = W_gate.shape
+    return torch.stack([W_gate.view(I // block, block, K), W_up.view(I // block, block, K)], dim=1).reshape(2 * I, K)
+
+
+def linear_swiglu(A: torch.Tensor, Asf: torch.Tensor, Wq: torch.Tensor, Wsf: torch.Tensor,
+                  inv_s_down: torch.Tensor | None, had_block_down: int = 32, *, Hq=None, Hsf=None, workspace=None):
+    """Gate/up linear (weights interleaved by interleave_gate_up, then prep_weights) followed by SwiGLU and
+    the down projection's activation quantization. Returns (Hq u8 [M, I/2], Hsf u8 tiled), the down
+    projection's A operand."""
+    N = Wq.shape[0]
+    K = Wq.shape[1] * 2
+    M = A.shape[0]
+    I = N // 2
+    dev = A.device
+    Hq = torch.empty(M, I // 2, dtype=torch.uint8, device=dev) if Hq is None else Hq
+    Hsf = torch.empty(max(sf_bytes(M, I), 16), dtype=torch.uint8, device=dev) if Hsf is None else Hsf
+    need = int(lib().macaq_linear_swiglu_workspace_bytes(M, N, K))
+    if workspace is None and need > 0:
+        workspace = _workspace(dev, need)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("macaq_linear_swiglu", lib().macaq_linear_swiglu(
+        _ptr(A), _ptr(Asf), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(inv_s_down), had_block_down, _ptr(Hq), _ptr(Hsf),
+        _ptr(workspace), ws_bytes, _stream(dev)))
+    return Hq, Hsf
+
+
+def swiglu_act_quant(GU: torch.Tensor, inv_s: torch.Tensor | None, had_block: int = 32, *, Hq=None, Hsf=None):
+    """MXFP4(silu(G) U diag(inv_s) H_b) from an fp32 gate/up output [M, 2I] (64-interleaved columns)."""
+    assert GU.dtype == torch.float32 and GU.dim() == 2
+    M, N = GU.shape
+    I = N // 2
+    dev = GU.device
+    Hq = torch.empty(M, I // 2, dtype=torch.uint8, device=dev) if Hq is None else Hq
+    Hsf = torch.empty(max(sf_bytes(M, I), 16), dtype=torch.uint8, device=dev) if Hsf is None else Hsf
+    _check("macaq_swiglu_act_quant", lib().macaq_swiglu_act_quant(
+        _ptr(GU), M, I, _ptr(inv_s), had_block, _ptr(Hq), _ptr(Hsf), _stream(dev)))
+    return Hq, Hsf
 
 
 def _out(M, N, out_dtype, dev, Y):

@@ -31,6 +31,7 @@
 #include "groups.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "swiglu.cuh"
 
 namespace macaq {
 
@@ -442,10 +443,36 @@ struct PairCfg {
     static constexpr int kThreads = kGemmThreads + 32;  // + a second producer warp for the scale factors
 };
 
+// Fused SwiGLU epilogue (kSwiglu = the down projection's Hadamard block b > 0): instead of writing
+// Y, each epilogue warp takes its 32 rows x (64 gate + 64 up columns) of the accumulator, which with
+// the 64-row gate/up interleave of the weights are intermediate channels [128 nt + 64 half, + 64),
+// and writes their SwiGLU, transformed and MXFP4-quantized (swiglu.cuh), as the down projection's A
+// operand: codes [M, I/2] and tiled SF. The gate/up output never reaches memory.
+template <int kB>
+__device__ __forceinline__ void epilogue_tile_pair_swiglu(uint32_t tmem, int warp, int lane, int32_t row0, int32_t nt,
+                                                          int64_t M, const SwigluOut &o, uint32_t accum_empty_addr) {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
+    uint32_t gv[64], uv[64];
+    tmem_ld64(taddr, gv);
+    tmem_ld64(taddr + 64, uv);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+    const int32_t c0 = nt * 128 + half * 64;
+    uint4 codes[2];
+    uint32_t E8[2];
+    swiglu_quant64<kB>(gv, uv, o.inv_s == nullptr ? nullptr : o.inv_s + c0, codes, E8);
+    store_swiglu64(o, static_cast<int64_t>(row0) + quarter * 32 + lane, M, c0, codes, E8);
+}
+
+template <int kSwiglu>
 __global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                       const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
-                      const __grid_constant__ CUtensorMap ymap, GemmArgs g, int sf_replica_boxes) {
+                      const __grid_constant__ CUtensorMap ymap, GemmArgs g, int sf_replica_boxes, SwigluOut so) {
     using C = PairCfg;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t dsmem[];
@@ -619,8 +646,12 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
             int leader_failed;
             asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(leader_failed) : "r"(leader_failed_addr) : "memory");
             if (failed || leader_failed) break;
-            epilogue_tile_pair(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128), static_cast<int32_t>(nt * 256),
-                               g.out_f32 != 0, &ymap, sEpi + (warp - 2) * 4096, empty_addr);
+            if constexpr (kSwiglu > 0)
+                epilogue_tile_pair_swiglu<kSwiglu>(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128),
+                                                   static_cast<int32_t>(nt), g.rows, so, empty_addr);
+            else
+                epilogue_tile_pair(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128), static_cast<int32_t>(nt * 256),
+                                   g.out_f32 != 0, &ymap, sEpi + (warp - 2) * 4096, empty_addr);
         }
         if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it
     }
@@ -724,6 +755,19 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
         return static_cast<uint32_t>(((static_cast<uint64_t>(u / g.gran) + 1) * C - 1) / chunks);
     };
 
+    // The weights do not depend on the previous kernel in the stream, and their loads need only this
+    // CTA's barriers: thread 0 requests the first stages' W' tiles and scale factors right after it
+    // has initialised the barriers, before TMEM is allocated (which may wait for the previous
+    // kernel's CTA on this SM to free its columns) and before the CTA-wide barrier.
+    auto load_w = [&](uint32_t u, int s) {
+        const uint32_t tile = u / num_kb;
+        const int kb = static_cast<int>(u - tile * num_kb);
+        if constexpr (kFused) mbar_arrive_expect_tx(&full_bar[s], 128 * kBKBytes + 4096);
+        else mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
+        tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
+        tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
+    };
+    const uint32_t pre = min(static_cast<uint32_t>(S), u_end > u_begin ? u_end - u_begin : 0u);
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], kFused ? 2 : 1);   // fused: the producer and the stage's quantizer warp
@@ -738,8 +782,9 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
         failed = 0;
         fence_mbar_init();
         prefetch_tensor_map(&wmap);
-        prefetch_tensor_map(&xmap);
         prefetch_tensor_map(&sfwmap);
+        for (uint32_t i = 0; i < pre; ++i) load_w(u_begin + i, static_cast<int>(i));
+        prefetch_tensor_map(&xmap);
         prefetch_tensor_map(&sfxmap);
     }
     if (warp == 1) {
@@ -767,16 +812,8 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ TMA producer
-            // The weights do not depend on the previous kernel in the stream: the first S stages' W'
-            // tiles and scale factors are requested before waiting for it; the activations after.
-            auto load_w = [&](uint32_t u, int s) {
-                const uint32_t tile = u / num_kb;
-                const int kb = static_cast<int>(u - tile * num_kb);
-                if constexpr (kFused) mbar_arrive_expect_tx(&full_bar[s], 128 * kBKBytes + 4096);
-                else mbar_arrive_expect_tx(&full_bar[s], (128 + mp) * kBKBytes + 8192);
-                tma_load_2d(sW(s), &wmap, &full_bar[s], kb * kBKBytes, static_cast<int32_t>(tile * 128));
-                tma_load_5d(sSfw(s), &sfwmap, &full_bar[s], 0, 0, 0, 0, static_cast<int32_t>(tile * kq + 2 * kb));
-            };
+            // The first `pre` stages' weights were requested at set-up; the activations may belong to
+            // the previous kernel, so they are requested after waiting for it.
             auto load_x = [&](uint32_t u, int s) {
                 const int kb = static_cast<int>(u % num_kb);
                 if constexpr (kFused) {
@@ -789,8 +826,6 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
                     tma_load_5d(sSfx(s), &sfxmap, &full_bar[s], 0, 0, 0, 0, 2 * kb);
                 }
             };
-            const uint32_t pre = min(static_cast<uint32_t>(S), u_end > u_begin ? u_end - u_begin : 0u);
-            for (uint32_t i = 0; i < pre; ++i) load_w(u_begin + i, static_cast<int>(i));
             griddep_wait();
             for (uint32_t i = 0; i < pre; ++i) load_x(u_begin + i, static_cast<int>(i));
             uint32_t j = pre;
@@ -965,18 +1000,26 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
                 if (s_last) {
+                    // the pieces are added in their fixed order (piece 0 first); four pieces x 16 rows of
+                    // loads are in flight per round trip to L2
                     float *base = g.partials + (static_cast<uint64_t>(tile) * g.max_pieces) * g.M * 128 + nl;
                     for (int m0 = 0; m0 < g.M; m0 += 16) {
                         float acc[16];
+                        for (int p0 = 0; p0 < npieces; p0 += 4) {
+                            float v[4][16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
-                        for (int p = 0; p < npieces; ++p) {  // 16 independent loads per piece: one round trip
-                            float v[16];
+                            for (int q = 0; q < 4; ++q)
 #pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                v[i] = (m0 + i < g.M) ? __ldcg(base + (static_cast<uint64_t>(p) * g.M + m0 + i) * 128) : 0.0f;
+                                for (int i = 0; i < 16; ++i)
+                                    v[q][i] = (p0 + q < npieces && m0 + i < g.M)
+                                                  ? __ldcg(base + (static_cast<uint64_t>(p0 + q) * g.M + m0 + i) * 128)
+                                                  : 0.0f;
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) acc[i] += v[i];
+                            for (int q = 0; q < 4; ++q) {
+                                if (p0 + q >= npieces) break;
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) acc[i] = (p0 + q == 0) ? v[q][i] : acc[i] + v[q][i];
+                            }
                         }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {

@@ -17,6 +17,7 @@
 
 #include "macaq.h"
 #include "gemm.cuh"
+#include "moe.cuh"
 #include "quant.cuh"
 
 namespace macaq {
@@ -205,16 +206,40 @@ macaq_status run_quant(int32_t b, const CUtensorMap &map, const QuantArgs &a, in
     }
 }
 
+template <int kB>
+macaq_status run_quant_gather_b(const QuantArgs &a, const GatherArgs &gx, int grid, cudaStream_t st) {
+    auto k = quant_gather_kernel<kB>;
+    const size_t smem = 2 * sizeof(int32_t) * (a.E + 1);
+    macaq_status s = set_smem(k, smem);
+    if (s != MACAQ_OK) return s;
+    return launch(k, dim3(grid), dim3(kQConsumers), smem, st, 1, a, gx);
+}
+
+macaq_status run_quant_gather(int32_t b, const QuantArgs &a, const GatherArgs &gx, int grid, cudaStream_t st) {
+    switch (b) {
+        case 1: return run_quant_gather_b<1>(a, gx, grid, st);
+        case 16: return run_quant_gather_b<16>(a, gx, grid, st);
+        case 32: return run_quant_gather_b<32>(a, gx, grid, st);
+        case 64: return run_quant_gather_b<64>(a, gx, grid, st);
+        case 128: return run_quant_gather_b<128>(a, gx, grid, st);
+        default: return MACAQ_ERR_UNSUPPORTED;
+    }
+}
+
+// row_index != nullptr: the gather form (activations only): output row m quantizes X row
+// row_index[m] of x_rows rows.
 macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, int32_t b, bool weight,
-                      const int32_t *offsets, int32_t E, uint8_t *q, uint8_t *sf, float *inv_s, cudaStream_t st) {
+                      const int32_t *offsets, int32_t E, uint8_t *q, uint8_t *sf, float *inv_s, cudaStream_t st,
+                      const int32_t *row_index = nullptr, int64_t x_rows = 0) {
     if (rows < 0 || K <= 0 || K % 128 != 0) return MACAQ_ERR_SHAPE;
     if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
     if (offsets != nullptr && (E < 1 || E > 16384)) return MACAQ_ERR_SHAPE;
     if (rows * (K / 32) >= (int64_t(1) << 31)) return MACAQ_ERR_SHAPE;
+    if (row_index != nullptr && (x_rows < 1 || x_rows * K >= (int64_t(1) << 40))) return MACAQ_ERR_SHAPE;
     if (rows == 0 && (inv_s == nullptr || mul == nullptr)) return MACAQ_OK;
     if (rows > 0 && (X == nullptr || q == nullptr || sf == nullptr)) return MACAQ_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(q) || !aligned16(sf) || !aligned16(mul) || !aligned16(inv_s) ||
-        !aligned16(offsets))
+        !aligned16(offsets) || !aligned16(row_index))
         return MACAQ_ERR_ALIGNMENT;
     DeviceInfo dev;
     macaq_status s = device_info(&dev);
@@ -237,6 +262,18 @@ macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, 
     a.E = offsets ? E : 1;
     a.wait_limit_ns = g_wait_limit_ns.load();
 
+    // CTAs: a multiple of the slab count, at most two per SM, no more than there are row tiles
+    uint32_t per_slab = (2u * dev.sms) / a.slabs;
+    if (per_slab > a.row_tiles) per_slab = a.row_tiles;
+    if (per_slab < 1) per_slab = 1;
+    const int grid = static_cast<int>(per_slab * a.slabs);
+    if (row_index != nullptr) {
+        GatherArgs gx;
+        gx.x = static_cast<const uint16_t *>(X);
+        gx.row_index = row_index;
+        gx.x_rows = x_rows;
+        return run_quant_gather(b, a, gx, grid, st);
+    }
     CUtensorMap map;
     std::memset(&map, 0, sizeof map);
     if (rows > 0) {
@@ -247,11 +284,6 @@ macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, 
         s = tensor_map(&map, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (s != MACAQ_OK) return s;
     }
-    // CTAs: a multiple of the slab count, at most two per SM, no more than there are row tiles
-    uint32_t per_slab = (2u * dev.sms) / a.slabs;
-    if (per_slab > a.row_tiles) per_slab = a.row_tiles;
-    if (per_slab < 1) per_slab = 1;
-    const int grid = static_cast<int>(per_slab * a.slabs);
     return weight ? run_quant<true>(b, map, a, grid, st) : run_quant<false>(b, map, a, grid, st);
 }
 
@@ -280,9 +312,19 @@ struct SkinnyPlan {
     size_t partial_bytes, count_bytes;
 };
 
-// Work split of the skinny GEMM on a device with `sms` SMs: equal contiguous unit ranges per CTA,
-// cut either anywhere (tiles split over CTAs, partial sums through the workspace) or on tile
-// boundaries (no partials), whichever moves fewer bytes per SM.
+// Work split of the skinny GEMM on a device with `sms` SMs: equal contiguous ranges of (weight tile,
+// K-block) units per CTA, cut either on tile boundaries (every CTA writes whole tiles) or anywhere
+// (a tile's pieces meet in the workspace and the CTA that finishes its last piece adds them). The
+// plan takes the cheapest of: whole tiles, and splits into at most 2, 3 or 4 pieces per tile on up
+// to all SMs, under a time model of the launch: streaming (the larger of the HBM time of all bytes
+// and one CTA's bytes at the rate a single SM sustains) plus, for splits, the final reduction (a
+// fence and atomic, then one L2 round trip per 16 rows, four pieces at a time).
+constexpr int kSkinnyMaxPiecesPerTile = 4;
+constexpr double kHbmBytesPerS = 6.0e12;      // sustained HBM read rate of a whole-GPU stream
+constexpr double kSmBytesPerS = 40.0e9;       // what one SM's TMA ring sustains on its own
+constexpr double kL2RoundTripS = 0.7e-6;      // one dependent L2 load round (reduction)
+constexpr double kReduceFixedS = 1.0e-6;      // fence + atomic + barrier before the reduction
+
 SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms, bool fused = false) {
     SkinnyPlan p{};
     p.mp = static_cast<int32_t>((M + 15) / 16 * 16);
@@ -290,31 +332,63 @@ SkinnyPlan skinny_plan(int64_t M, int64_t N, int64_t K, int sms, bool fused = fa
     const uint32_t num_kb = static_cast<uint32_t>(K / 256);
     p.units = p.tiles * num_kb;
     const double w_bytes = static_cast<double>(N) * K * 0.53125;
-    const uint32_t whole_ctas = p.tiles < static_cast<uint32_t>(sms) ? p.tiles : static_cast<uint32_t>(sms);
-    const double whole_cost = w_bytes / whole_ctas * ((p.tiles + whole_ctas - 1) / whole_ctas) / (static_cast<double>(p.tiles) / whole_ctas);
-    const uint32_t split_ctas = p.units < static_cast<uint32_t>(sms) ? p.units : static_cast<uint32_t>(sms);
-    const double pieces = p.tiles + split_ctas;  // every range boundary adds at most one piece
-    // per-SM bytes, plus the partial traffic (write, read) and the serial cross-CTA reduction at the
-    // end (a fence, an atomic and a round trip: about what an SM streams in 2.5 us)
-    const double split_cost = (w_bytes + 2.0 * pieces * M * 128 * 4) / split_ctas + 125.0e3;
-    const bool split = split_cost < whole_cost;
-    p.gran = split ? 1 : num_kb;
-    p.ctas = split ? split_ctas : whole_ctas;
-    const uint32_t chunks = p.units / p.gran;
-    int max_pieces = 1;
-    for (uint32_t t = 0; t < p.tiles && split; ++t) {
-        const uint64_t u0 = static_cast<uint64_t>(t) * num_kb, u1 = u0 + num_kb - 1;
-        const uint64_t c0 = ((u0 / p.gran + 1) * p.ctas - 1) / chunks, c1 = ((u1 / p.gran + 1) * p.ctas - 1) / chunks;
-        const int np = static_cast<int>(c1 - c0 + 1);
-        if (np > max_pieces) max_pieces = np;
+    const double tile_bytes = w_bytes / p.tiles;
+    // pieces of the tile cut most often when `ctas` equal ranges of unit granularity `gran` are used
+    auto pieces_of = [&](uint32_t ctas, uint32_t gran) {
+        const uint32_t chunks = p.units / gran;
+        int mx = 1;
+        for (uint32_t t = 0; t < p.tiles; ++t) {
+            const uint64_t u0 = static_cast<uint64_t>(t) * num_kb, u1 = u0 + num_kb - 1;
+            const uint64_t c0 = ((u0 / gran + 1) * ctas - 1) / chunks, c1 = ((u1 / gran + 1) * ctas - 1) / chunks;
+            mx = std::max(mx, static_cast<int>(c1 - c0 + 1));
+        }
+        return mx;
+    };
+    // whole tiles
+    const uint32_t whole_ctas = std::min<uint32_t>(p.tiles, static_cast<uint32_t>(sms));
+    const double whole_per_cta = tile_bytes * ((p.tiles + whole_ctas - 1) / whole_ctas);
+    double best = std::max(w_bytes / kHbmBytesPerS, whole_per_cta / kSmBytesPerS);
+    p.gran = num_kb;
+    p.ctas = whole_ctas;
+    p.max_pieces = 1;
+    const uint64_t most = std::min<uint64_t>(static_cast<uint64_t>(sms), p.units);
+    const uint64_t cands[3] = {std::min<uint64_t>(most, 2ull * p.tiles), std::min<uint64_t>(most, 3ull * p.tiles), most};
+    for (uint64_t c : cands) {
+        const uint32_t ctas = static_cast<uint32_t>(c);
+        if (ctas <= whole_ctas) continue;
+        const int pieces = pieces_of(ctas, 1);
+        if (pieces > kSkinnyMaxPiecesPerTile) continue;
+        const double part_bytes = 2.0 * pieces * p.tiles * M * 128 * 4;
+        const double t = std::max((w_bytes + part_bytes) / kHbmBytesPerS, w_bytes / ctas / kSmBytesPerS) +
+                         kReduceFixedS + ((M + 15) / 16) * ((pieces + 3) / 4) * kL2RoundTripS;
+        if (t < best) {
+            best = t;
+            p.gran = 1;
+            p.ctas = ctas;
+            p.max_pieces = pieces;
+        }
     }
-    p.max_pieces = max_pieces;
-    p.partial_bytes = split ? static_cast<size_t>(p.tiles) * max_pieces * static_cast<size_t>(M) * 128 * 4 : 0;
+    const bool split = p.gran == 1;
+    p.partial_bytes = split ? static_cast<size_t>(p.tiles) * p.max_pieces * static_cast<size_t>(M) * 128 * 4 : 0;
     p.count_bytes = kCountRegion;
     p.ok = static_cast<size_t>(p.tiles) * 4 <= kCountRegion;
     const int smem_budget = 232448 - 1024 - 1024 - skinny_stage_bytes_y(p.mp);  // minus slack, static data, Y staging
     int st = smem_budget / (fused ? skinny_stage_bytes_fused(p.mp) : skinny_stage_bytes(p.mp));
     p.stages = st > kSkinnyMaxStages ? kSkinnyMaxStages : st;
+    return p;
+}
+
+// skinny_plan() memoised per (shape, SM count, form): it runs on every call.
+SkinnyPlan skinny_plan_cached(int64_t M, int64_t N, int64_t K, int sms, bool fused = false) {
+    static std::mutex mu;
+    static std::map<std::tuple<int64_t, int64_t, int64_t, int, bool>, SkinnyPlan> cache;
+    const auto key = std::make_tuple(M, N, K, sms, fused);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    const SkinnyPlan p = skinny_plan(M, N, K, sms, fused);
+    if (cache.size() > 4096) cache.clear();
+    cache.emplace(key, p);
     return p;
 }
 
@@ -338,7 +412,7 @@ macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, i
                         int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
                         size_t ws_bytes, int sms, cudaStream_t st, size_t clear_counts = 0) {
     const bool fused = fused_b > 0;
-    const SkinnyPlan p = skinny_plan(M, N, K, sms, fused);
+    const SkinnyPlan p = skinny_plan_cached(M, N, K, sms, fused);
     if (!p.ok) return MACAQ_ERR_SHAPE;
     // the in-kernel quantizer warps take the stages in turn, four at a time: a stage count that is
     // not a multiple of four would give one stage to two warps at different phases
@@ -405,6 +479,76 @@ macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, i
     }
 }
 
+// The dense GEMM on 2-SM pairs (M > 128, N % 256 == 0, K % 256 == 0). swiglu_b > 0 selects the fused
+// SwiGLU epilogue (the down projection's quantized input goes to `so` instead of Y).
+template <int kSwiglu>
+macaq_status launch_pair(const CUtensorMap &amap, const CUtensorMap &bmap, const CUtensorMap &sfamap,
+                         const CUtensorMap &sfbmap, const CUtensorMap &ymap, const GemmArgs &g, int replica_boxes,
+                         const SwigluOut &so, unsigned pairs, cudaStream_t st) {
+    auto k = gemm_mxf4_pair_kernel<kSwiglu>;
+    macaq_status s = set_smem(k, PairCfg::kSmemBytes);
+    if (s != MACAQ_OK) return s;
+    return launch(k, dim3(2 * pairs), dim3(PairCfg::kThreads), PairCfg::kSmemBytes, st, 2, amap, bmap, sfamap, sfbmap,
+                  ymap, g, replica_boxes, so);
+}
+
+macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_t N, int64_t K, const uint8_t *Wq,
+                      const uint8_t *Wsf, void *Y, int32_t out_dtype, const GemmArgs &g, int32_t swiglu_b,
+                      const SwigluOut &so, int sms, cudaStream_t st) {
+    macaq_status s;
+    CUtensorMap amap, bmap, sfamap, sfbmap;
+    s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s == MACAQ_OK)
+        s = tensor_map_2d(&bmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    // replica views of the SF buffers: (128 B, half h, 8-row group i, 128x4 tile c); for A the
+    // halves are the K-block's two tiles (512 B apart), for B the two 128-row tiles of the
+    // 256-row N tile (K/128 tiles apart)
+    const uint64_t kq = static_cast<uint64_t>(K / 128);
+    // one 4 KB box holding all four replicas needs a zero-stride replica dimension; if the driver
+    // refuses that view, four 1 KB boxes (one replica each) are used instead
+    int replica_boxes = 1;
+    if (s == MACAQ_OK) {
+        const uint64_t da[5] = {128, 2, 4, 4, macaq_sf_bytes(rows, K) / 512};
+        const uint64_t sa[4] = {512, 128, 0, 512};
+        const uint64_t db[5] = {128, 2, 4, 4, macaq_sf_bytes(N, K) / 512};
+        const uint64_t sb[4] = {kq * 512, 128, 0, 512};
+        const uint32_t box[5] = {128, 2, 4, 4, 1};
+        if (tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, da, sa, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK ||
+            tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, db, sb, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK) {
+            replica_boxes = 4;
+            const uint64_t da4[4] = {128, 2, 4, macaq_sf_bytes(rows, K) / 512};
+            const uint64_t sa4[3] = {512, 128, 512};
+            const uint64_t db4[4] = {128, 2, 4, macaq_sf_bytes(N, K) / 512};
+            const uint64_t sb4[3] = {kq * 512, 128, 512};
+            const uint32_t box4[4] = {128, 2, 4, 1};
+            s = tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, da4, sa4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (s == MACAQ_OK)
+                s = tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, db4, sb4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
+        }
+    }
+    // Y in 32-row x 128-byte boxes, 128-byte swizzled (the epilogue's staging layout)
+    CUtensorMap ymap = amap;   // the fused SwiGLU epilogue writes no Y (the map is not used)
+    if (s == MACAQ_OK && swiglu_b == 0) {
+        const bool f32 = out_dtype == MACAQ_OUT_F32;
+        s = tensor_map_2d(&ymap, Y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, rows,
+                          N * (f32 ? 4 : 2), f32 ? 32 : 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (s != MACAQ_OK) return s;
+    const int64_t tiles = ((rows + 255) / 256) * (N / 256);
+    const int64_t max_pairs = sms / 2;
+    const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
+    switch (swiglu_b) {
+        case 0: return launch_pair<0>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
+        case 1: return launch_pair<1>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
+        case 16: return launch_pair<16>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
+        case 32: return launch_pair<32>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
+        case 64: return launch_pair<64>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
+        default: return MACAQ_ERR_UNSUPPORTED;
+    }
+}
+
 macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, int32_t E, int64_t rows, int64_t N,
                   int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
                   size_t ws_bytes, cudaStream_t st) {
@@ -423,7 +567,7 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
     if (s != MACAQ_OK) return s;
 
     if (offsets == nullptr && rows <= kSkinnyMaxM && K % 256 == 0 && workspace != nullptr &&
-        skinny_plan(rows, N, K, dev.sms).ok)
+        skinny_plan_cached(rows, N, K, dev.sms).ok)
         return run_skinny(A, Asf, nullptr, 0, rows, N, K, Wq, Wsf, Y, out_dtype, workspace, ws_bytes, dev.sms, st);
 
     const int BN = (N % 256 == 0) ? 256 : 128;
@@ -443,55 +587,7 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
     g.bsf_stride = macaq_sf_bytes(N, K);
     g.wait_limit_ns = g_wait_limit_ns.load();
 
-    if (pair) {
-        CUtensorMap amap, bmap, sfamap, sfbmap;
-        s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, 128,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
-        if (s == MACAQ_OK)
-            s = tensor_map_2d(&bmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128,
-                              CU_TENSOR_MAP_SWIZZLE_128B);
-        // replica views of the SF buffers: (128 B, half h, 8-row group i, 128x4 tile c); for A the
-        // halves are the K-block's two tiles (512 B apart), for B the two 128-row tiles of the
-        // 256-row N tile (K/128 tiles apart)
-        const uint64_t kq = static_cast<uint64_t>(K / 128);
-        // one 4 KB box holding all four replicas needs a zero-stride replica dimension; if the driver
-        // refuses that view, four 1 KB boxes (one replica each) are used instead
-        int replica_boxes = 1;
-        if (s == MACAQ_OK) {
-            const uint64_t da[5] = {128, 2, 4, 4, macaq_sf_bytes(rows, K) / 512};
-            const uint64_t sa[4] = {512, 128, 0, 512};
-            const uint64_t db[5] = {128, 2, 4, 4, macaq_sf_bytes(N, K) / 512};
-            const uint64_t sb[4] = {kq * 512, 128, 0, 512};
-            const uint32_t box[5] = {128, 2, 4, 4, 1};
-            if (tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, da, sa, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK ||
-                tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, db, sb, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK) {
-                replica_boxes = 4;
-                const uint64_t da4[4] = {128, 2, 4, macaq_sf_bytes(rows, K) / 512};
-                const uint64_t sa4[3] = {512, 128, 512};
-                const uint64_t db4[4] = {128, 2, 4, macaq_sf_bytes(N, K) / 512};
-                const uint64_t sb4[3] = {kq * 512, 128, 512};
-                const uint32_t box4[4] = {128, 2, 4, 1};
-                s = tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, da4, sa4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
-                if (s == MACAQ_OK)
-                    s = tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, db4, sb4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
-            }
-        }
-        // Y in 32-row x 128-byte boxes, 128-byte swizzled (the epilogue's staging layout)
-        CUtensorMap ymap;
-        if (s == MACAQ_OK) {
-            const bool f32 = out_dtype == MACAQ_OUT_F32;
-            s = tensor_map_2d(&ymap, Y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, rows,
-                              N * (f32 ? 4 : 2), f32 ? 32 : 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
-        }
-        if (s != MACAQ_OK) return s;
-        const int64_t tiles = ((rows + 255) / 256) * (N / 256);
-        const int64_t max_pairs = dev.sms / 2;
-        const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
-        s = set_smem(gemm_mxf4_pair_kernel, PairCfg::kSmemBytes);
-        if (s != MACAQ_OK) return s;
-        return launch(gemm_mxf4_pair_kernel, dim3(2 * pairs), dim3(PairCfg::kThreads), PairCfg::kSmemBytes, st, 2, amap,
-                      bmap, sfamap, sfbmap, ymap, g, replica_boxes);
-    }
+    if (pair) return run_pair(A, Asf, rows, N, K, Wq, Wsf, Y, out_dtype, g, 0, SwigluOut{}, dev.sms, st);
 
     CUtensorMap amap, bmap;
     s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, kBM,
@@ -541,7 +637,7 @@ macaq_status linear_fixed_scratch(const uint8_t *A, const uint8_t *Asf, int64_t 
     DeviceInfo dev;
     macaq_status s = device_info(&dev);
     if (s != MACAQ_OK) return s;
-    const SkinnyPlan p = skinny_plan(M, N, K, dev.sms);
+    const SkinnyPlan p = skinny_plan_cached(M, N, K, dev.sms);
     if (!p.ok) return gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, nullptr, 0, st);
     if (p.partial_bytes + p.count_bytes > MACAQ_FIXED_SCRATCH_BYTES) return MACAQ_ERR_WORKSPACE;
     void *scratch = nullptr;
@@ -568,7 +664,7 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
     FusedLayout f{};
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     if (E == 0 && M >= 1 && M <= kSkinnyMaxM && K % 256 == 0) {
-        const SkinnyPlan p = skinny_plan(M, N, K, sms, M <= kSkinnyFusedMaxM);
+        const SkinnyPlan p = skinny_plan_cached(M, N, K, sms, M <= kSkinnyFusedMaxM);
         if (p.ok) {
             f.gemm_ws = up(p.count_bytes + p.partial_bytes);
             // the quantizer warps need a stage count that is a multiple of four (run_skinny checks it)
@@ -613,6 +709,132 @@ macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const in
                 f.gemm_ws > 0 ? ws : nullptr, f.gemm_ws, st);
 }
 
+// ------------------------------------------------------------------------ SwiGLU -> down-projection input
+bool valid_swiglu_block(int32_t b) { return b == 1 || b == 16 || b == 32 || b == 64; }
+
+template <int kB>
+macaq_status launch_swiglu_quant(const float *gu, int64_t M, const SwigluOut &o, int sms, cudaStream_t st) {
+    const int64_t items = static_cast<int64_t>(o.rows_sf) * (o.I / 64);
+    int64_t blocks = (items + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    if (blocks > cap) blocks = cap;
+    return launch(swiglu_quant_kernel<kB>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 1, gu, M, o);
+}
+
+// H' = MXFP4(swiglu(G, U) diag(inv_s) H_b) from a gate/up output in memory (fp32 [M, 2I], 64-interleaved).
+macaq_status swiglu_quant(const float *gu, int64_t M, int64_t I, const float *inv_s, int32_t b, uint8_t *hq, uint8_t *hsf,
+                          cudaStream_t st) {
+    if (M < 0 || I <= 0 || I % 128 != 0 || M >= (int64_t(1) << 31) || I >= (int64_t(1) << 30)) return MACAQ_ERR_SHAPE;
+    if (!valid_swiglu_block(b)) return MACAQ_ERR_UNSUPPORTED;
+    if (M == 0) return MACAQ_OK;
+    if (gu == nullptr || hq == nullptr || hsf == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(gu) || !aligned16(inv_s) || !aligned16(hq) || !aligned16(hsf)) return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+    SwigluOut o{inv_s, hq, hsf, static_cast<int32_t>(I), static_cast<int32_t>((M + 127) / 128 * 128)};
+    switch (b) {
+        case 1: return launch_swiglu_quant<1>(gu, M, o, dev.sms, st);
+        case 16: return launch_swiglu_quant<16>(gu, M, o, dev.sms, st);
+        case 32: return launch_swiglu_quant<32>(gu, M, o, dev.sms, st);
+        default: return launch_swiglu_quant<64>(gu, M, o, dev.sms, st);
+    }
+}
+
+// Whether the gate/up GEMM of these sizes runs the fused epilogue (2-SM pair kernel), and otherwise
+// the workspace of the two-step form: the skinny GEMM's region (when it runs), then the fp32 gate/up
+// output.
+struct SwigluLayout {
+    bool fused;
+    size_t gemm_ws, gu_off, total;
+};
+
+SwigluLayout swiglu_layout(int64_t M, int64_t N, int64_t K, int sms) {
+    SwigluLayout l{};
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    l.fused = M > kSkinnyMaxM && N % 256 == 0 && K % 256 == 0;
+    if (l.fused) return l;
+    if (M >= 1 && M <= kSkinnyMaxM && K % 256 == 0) {
+        const SkinnyPlan p = skinny_plan_cached(M, N, K, sms);
+        if (p.ok) l.gemm_ws = up(p.count_bytes + p.partial_bytes);
+    }
+    l.gu_off = std::max(l.gemm_ws, up(kCountRegion));
+    l.total = l.gu_off + up(static_cast<size_t>(M) * static_cast<size_t>(N) * 4);
+    return l;
+}
+
+macaq_status linear_swiglu(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K, const uint8_t *Wq,
+                           const uint8_t *Wsf, const float *inv_s, int32_t b, uint8_t *hq, uint8_t *hsf, void *workspace,
+                           size_t ws_bytes, cudaStream_t st) {
+    if (M < 0 || N <= 0 || N % 256 != 0 || K <= 0 || K % 128 != 0) return MACAQ_ERR_SHAPE;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return MACAQ_ERR_SHAPE;
+    if (!valid_swiglu_block(b)) return MACAQ_ERR_UNSUPPORTED;
+    if (M == 0) return MACAQ_OK;
+    if (A == nullptr || Asf == nullptr || Wq == nullptr || Wsf == nullptr || hq == nullptr || hsf == nullptr)
+        return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(Asf) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(inv_s) || !aligned16(hq) ||
+        !aligned16(hsf) || !aligned16(workspace))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+    const SwigluLayout l = swiglu_layout(M, N, K, dev.sms);
+    const int64_t I = N / 2;
+    if (l.fused) {
+        GemmArgs g{};
+        g.asf = Asf;
+        g.bsf = Wsf;
+        g.y = nullptr;
+        g.offsets = nullptr;
+        g.rows = M;
+        g.N = static_cast<int32_t>(N);
+        g.K = static_cast<int32_t>(K);
+        g.E = 1;
+        g.out_f32 = 0;
+        g.bsf_stride = macaq_sf_bytes(N, K);
+        g.wait_limit_ns = g_wait_limit_ns.load();
+        SwigluOut o{inv_s, hq, hsf, static_cast<int32_t>(I), static_cast<int32_t>((M + 127) / 128 * 128)};
+        return run_pair(A, Asf, M, N, K, Wq, Wsf, nullptr, MACAQ_OUT_BF16, g, b, o, dev.sms, st);
+    }
+    if (workspace == nullptr || ws_bytes < l.total) return MACAQ_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *gu = reinterpret_cast<float *>(ws + l.gu_off);
+    s = gemm(A, Asf, nullptr, 1, M, N, K, Wq, Wsf, gu, MACAQ_OUT_F32, l.gemm_ws > 0 ? ws : nullptr, l.gemm_ws, st);
+    if (s != MACAQ_OK) return s;
+    return swiglu_quant(gu, M, I, inv_s, b, hq, hsf, st);
+}
+
+// ------------------------------------------------------------------------ MoE combine
+macaq_status moe_combine(const void *Y, int64_t y_rows, int64_t N, const int32_t *pos, const float *w, int64_t T,
+                         int32_t topk, void *out, int32_t out_dtype, cudaStream_t st) {
+    if (y_rows < 0 || N <= 0 || N % 8 != 0 || T < 0 || topk < 1 || topk > 1024) return MACAQ_ERR_SHAPE;
+    if (N >= (int64_t(1) << 31) || T * topk >= (int64_t(1) << 40)) return MACAQ_ERR_SHAPE;
+    if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
+    if (T == 0) return MACAQ_OK;
+    if ((Y == nullptr && y_rows > 0) || pos == nullptr || w == nullptr || out == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(Y) || !aligned16(out) || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+        (reinterpret_cast<uintptr_t>(w) & 3u))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+    CombineArgs c;
+    c.y = static_cast<const uint16_t *>(Y);
+    c.pos = pos;
+    c.w = w;
+    c.out = out;
+    c.y_rows = y_rows;
+    c.T = T;
+    c.topk = topk;
+    c.N = static_cast<int32_t>(N);
+    c.out_f32 = out_dtype == MACAQ_OUT_F32;
+    const int64_t threads = T * (N / 8);
+    int64_t blocks = (threads + kCombineThreads - 1) / kCombineThreads;
+    const int64_t cap = static_cast<int64_t>(dev.sms) * 8;   // 8 resident CTAs per SM, grid-stride beyond
+    if (blocks > cap) blocks = cap;
+    return launch(moe_combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kCombineThreads), 0, st, 1, c);
+}
+
 }  // namespace macaq
 
 // ============================================================================ C ABI
@@ -649,7 +871,7 @@ size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t E) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 0;
-    const macaq::SkinnyPlan p = macaq::skinny_plan(M, N, K, sms);
+    const macaq::SkinnyPlan p = macaq::skinny_plan_cached(M, N, K, sms);
     return p.ok ? p.partial_bytes + p.count_bytes : 0;
 }
 
@@ -673,6 +895,41 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
                              macaq_stream_t stream) {
     return macaq::quantize(X, inv_s, M, K, had_block, false, group_offsets, E, Xq, Xsf, nullptr,
                            static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_act_quant_gather(const void *X, int64_t x_rows, const int32_t *row_index, const float *inv_s,
+                                    int64_t M, int64_t K, int32_t had_block, const int32_t *group_offsets, int32_t E,
+                                    uint8_t *Xq, uint8_t *Xsf, macaq_stream_t stream) {
+    if (row_index == nullptr && M > 0) return MACAQ_ERR_INVALID_ARG;
+    if (M == 0) return macaq::quantize(X, inv_s, 0, K, had_block, false, group_offsets, E, Xq, Xsf, nullptr,
+                                       static_cast<cudaStream_t>(stream));
+    return macaq::quantize(X, inv_s, M, K, had_block, false, group_offsets, E, Xq, Xsf, nullptr,
+                           static_cast<cudaStream_t>(stream), row_index, x_rows);
+}
+
+size_t macaq_linear_swiglu_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N <= 0 || N % 256 != 0 || K <= 0 || K % 128 != 0) return 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return macaq::swiglu_layout(M, N, K, sms).total;
+}
+
+macaq_status macaq_linear_swiglu(const uint8_t *A, const uint8_t *Asf, int64_t M, int64_t N, int64_t K,
+                                 const uint8_t *Wq, const uint8_t *Wsf, const float *inv_s_down, int32_t had_block_down,
+                                 uint8_t *Hq, uint8_t *Hsf, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
+    return macaq::linear_swiglu(A, Asf, M, N, K, Wq, Wsf, inv_s_down, had_block_down, Hq, Hsf, workspace, ws_bytes,
+                                static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_swiglu_act_quant(const float *GU, int64_t M, int64_t I, const float *inv_s, int32_t had_block,
+                                    uint8_t *Hq, uint8_t *Hsf, macaq_stream_t stream) {
+    return macaq::swiglu_quant(GU, M, I, inv_s, had_block, Hq, Hsf, static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_moe_combine(const void *Y, int64_t y_rows, int64_t N, const int32_t *pos, const float *weights,
+                               int64_t T, int32_t topk, void *out, int32_t out_dtype, macaq_stream_t stream) {
+    return macaq::moe_combine(Y, y_rows, N, pos, weights, T, topk, out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
 macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M, int64_t N,

@@ -102,6 +102,11 @@ __device__ __forceinline__ void load_mul(const float *mul, uint64_t (&mv)[16]) {
 // pairs, then its MXFP4 encoding: the 16 code bytes (even k in the low nibble) and the E8M0
 // exponent. For b >= 64 the group is paired with the groups of lanes lane ^ 1 (and lane ^ 2), which
 // hold the next groups of the same row: the whole warp calls it together.
+// OCP MX v1.0 encoding of one 32-element group held as 16 packed fp32 pairs: the shared E8M0
+// exponent E = clamp(floor(log2 amax) - 2 + 127, 0, 254) read from the exponent field of amax, and
+// the 32 E2M1 codes of v * 2^(127 - E) (round to nearest even, saturating), two per byte.
+__device__ __forceinline__ void mx_encode_group(const uint64_t (&p)[16], uint4 &packed, uint32_t &E8);
+
 template <int kB, bool kWeight>
 __device__ __forceinline__ void transform_quantize_group(uint64_t (&p)[16], uint4 &packed, uint32_t &E8) {
     if constexpr (kB > 1) {
@@ -114,7 +119,10 @@ __device__ __forceinline__ void transform_quantize_group(uint64_t (&p)[16], uint
             for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], inv_b);
         }
     }
+    mx_encode_group(p, packed, E8);
+}
 
+__device__ __forceinline__ void mx_encode_group(const uint64_t (&p)[16], uint4 &packed, uint32_t &E8) {
     float mx[16];  // max |v| as a tree: short dependency chains
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -148,6 +156,50 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&raw)[4], uint64_t (
         p[4 * i + 1] = pk2(__uint_as_float(raw[i].y << 16), __uint_as_float(raw[i].y & 0xFFFF0000u));
         p[4 * i + 2] = pk2(__uint_as_float(raw[i].z << 16), __uint_as_float(raw[i].z & 0xFFFF0000u));
         p[4 * i + 3] = pk2(__uint_as_float(raw[i].w << 16), __uint_as_float(raw[i].w & 0xFFFF0000u));
+    }
+}
+
+// The rest of one group's work once its 32 inputs are fp32 pairs in registers: the per-channel
+// multiply (mv, when a.mul is set), Hadamard and MXFP4 (transform_quantize_group), the 16 code bytes
+// of row m, and the E8M0 byte, which lanes 4i..4i+3 (scale columns 4c..4c+3 of one row) combine into
+// one 32-bit store in the tiled layout. e < 0 marks a row outside every group: nothing is stored.
+// The whole warp calls it together (shuffles).
+template <int kB, bool kWeight>
+__device__ __forceinline__ void quantize_store_group(uint64_t (&p)[16], const uint64_t (&mv)[16], const QuantArgs &a,
+                                                     int e, uint32_t m, uint32_t g, const int32_t *s_off,
+                                                     const int32_t *s_tb, int lane) {
+    if (a.mul != nullptr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
+    }
+    uint4 packed;
+    uint32_t E8;
+    transform_quantize_group<kB, kWeight>(p, packed, E8);
+    const bool store = e >= 0;
+    if (store) *reinterpret_cast<uint4 *>(a.q + static_cast<uint64_t>(m) * (a.K / 2) + g * 16) = packed;
+    const uint32_t b1 = __shfl_down_sync(0xffffffffu, E8, 1);
+    const uint32_t b2 = __shfl_down_sync(0xffffffffu, E8, 2);
+    const uint32_t b3 = __shfl_down_sync(0xffffffffu, E8, 3);
+    if (store && (lane & 3) == 0) {
+        const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + (m - static_cast<uint32_t>(s_off[e]));
+        *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, g, a.kg >> 2)) = E8 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+}
+
+// Zeroes the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1): groups are
+// dealt to the CTAs in turn, one warp per padding row, lanes over the 32-bit words (4 scale columns
+// each) of that row.
+__device__ __forceinline__ void zero_sf_padding(const QuantArgs &a, const int32_t *s_off, const int32_t *s_tb, int warp,
+                                                int lane, int warps) {
+    const uint32_t kq = a.kg >> 2;
+    for (int e = blockIdx.x; e < a.E; e += gridDim.x) {
+        const uint32_t me = static_cast<uint32_t>(s_off[e + 1] - s_off[e]);
+        const uint32_t nt = static_cast<uint32_t>(s_tb[e + 1] - s_tb[e]);
+        for (uint32_t pr = me + warp; pr < nt * 128; pr += warps) {
+            const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + pr;
+            for (uint32_t w = lane; w < kq; w += 32)
+                *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, 4 * w, kq)) = 0u;
+        }
     }
 }
 
@@ -239,47 +291,92 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[s]);
-            if (a.mul != nullptr) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
-            }
-
-            uint4 packed;
-            uint32_t E8;
-            transform_quantize_group<kB, kWeight>(p, packed, E8);
-            const bool store = e >= 0;
-            if (store)
-                *reinterpret_cast<uint4 *>(a.q + static_cast<uint64_t>(m) * (a.K / 2) + g * 16) = packed;
-
-            // lanes 4i..4i+3 hold scale columns 4c..4c+3 of one row: one 32-bit store
-            const uint32_t b1 = __shfl_down_sync(0xffffffffu, E8, 1);
-            const uint32_t b2 = __shfl_down_sync(0xffffffffu, E8, 2);
-            const uint32_t b3 = __shfl_down_sync(0xffffffffu, E8, 3);
-            if (store && (lane & 3) == 0) {
-                const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + (m - static_cast<uint32_t>(s_off[e]));
-                *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, g, a.kg >> 2)) =
-                    E8 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-            }
+            quantize_store_group<kB, kWeight>(p, mv, a, e, m, g, s_off, s_tb, lane);
         }
     }
 
-    // zero the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1):
-    // one warp per padding row, lanes over the 32-bit words (4 scale columns each) of that row
-    const uint32_t kq = a.kg >> 2;
-    for (int e = blockIdx.x; e < a.E; e += gridDim.x) {
-        const uint32_t me = static_cast<uint32_t>(s_off[e + 1] - s_off[e]);
-        const uint32_t nt = static_cast<uint32_t>(s_tb[e + 1] - s_tb[e]);
-        for (uint32_t pr = me + warp; pr < nt * 128; pr += kQThreads / 32) {
-            const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + pr;
-            for (uint32_t w = lane; w < kq; w += 32)
-                *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, 4 * w, kq)) = 0u;
-        }
-    }
+    zero_sf_padding(a, s_off, s_tb, warp, lane, kQThreads / 32);
 
     if (kWeight && a.inv_s != nullptr && a.mul != nullptr) {
         for (uint32_t k = blockIdx.x * blockDim.x + tid; k < a.K; k += gridDim.x * blockDim.x)
             a.inv_s[k] = __fdiv_rn(1.0f, a.mul[k]);
     }
+}
+
+// Activation quantization with a row gather (MoE dispatch): output row m is the transform and MXFP4
+// of input row row_index[m] of X (x_rows rows), so the caller never materialises the expert-sorted
+// copy of the activations. Same work split as quant_kernel (column slabs, contiguous runs of row
+// tiles, multipliers in registers per expert) and the same per-group arithmetic; the gathered rows
+// are not contiguous, so each thread loads its 64-byte group straight from global memory (a warp's
+// lanes read one or more whole 512- to 2048-byte row segments), one row tile ahead of the one it
+// quantizes. Index values outside [0, x_rows) are clamped into it (no access leaves X; the result
+// for such a row is that of the clamped row).
+// Source: glonce.com page on MACaQ, paragraph 5 (grouped matmul for mixture-of-experts layers).
+struct GatherArgs {
+    const uint16_t *x;         // bf16 [x_rows, K]
+    const int32_t *row_index;  // [rows]
+    int64_t x_rows;
+};
+
+__device__ __forceinline__ void load_group_global(const uint16_t *src, uint4 (&raw)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(raw[i].x), "=r"(raw[i].y), "=r"(raw[i].z), "=r"(raw[i].w)
+                     : "l"(src + 8 * i));
+}
+
+template <int kB>
+__global__ void __launch_bounds__(kQConsumers, 2) quant_gather_kernel(QuantArgs a, GatherArgs gx) {
+    extern __shared__ uint8_t dsmem[];
+    int32_t *s_off = reinterpret_cast<int32_t *>(dsmem);
+    int32_t *s_tb = s_off + (a.E + 1);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const uint32_t slab = blockIdx.x % a.slabs;
+    const uint32_t ctas_per_slab = gridDim.x / a.slabs;
+    const uint32_t c_in_slab = blockIdx.x / a.slabs;
+    const uint32_t rt_begin = static_cast<uint32_t>(static_cast<uint64_t>(a.row_tiles) * c_in_slab / ctas_per_slab);
+    const uint32_t rt_end = static_cast<uint32_t>(static_cast<uint64_t>(a.row_tiles) * (c_in_slab + 1) / ctas_per_slab);
+    griddep_wait();  // X, the indices, the offsets and the outputs may belong to the previous kernel
+    load_group_layout(a.offsets, a.E, a.rows, s_off, s_tb);  // contains __syncthreads
+    griddep_launch_dependents();
+
+    const uint32_t gc = tid & (a.slab_groups - 1);
+    const uint32_t r_in = tid >> a.slab_shift;
+    const uint32_t g = slab * a.slab_groups + gc;
+    auto fetch = [&](uint32_t rt, uint4 (&raw)[4]) {
+        const uint32_t m = rt * a.tile_rows + r_in;
+        if (m < a.rows) {
+            int64_t src = gx.row_index[m];
+            src = src < 0 ? 0 : (src >= gx.x_rows ? gx.x_rows - 1 : src);
+            load_group_global(gx.x + static_cast<uint64_t>(src) * a.K + g * 32, raw);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    uint64_t mv[16];
+    int cur_e = -1;
+    uint4 next[4];
+    if (rt_begin < rt_end) fetch(rt_begin, next);
+    for (uint32_t rt = rt_begin; rt < rt_end; ++rt) {
+        uint4 raw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) raw[i] = next[i];
+        if (rt + 1 < rt_end) fetch(rt + 1, next);   // the next tile's loads are in flight meanwhile
+        const uint32_t m = rt * a.tile_rows + r_in;
+        const int e = m < a.rows ? find_group(s_off, a.E, m) : -1;
+        if (a.mul != nullptr && e != cur_e && e >= 0) {
+            load_mul(a.mul + static_cast<uint64_t>(e) * a.K + g * 32, mv);
+            cur_e = e;
+        }
+        uint64_t p[16];
+        unpack_bf16x32(raw, p);
+        quantize_store_group<kB, false>(p, mv, a, e, m, g, s_off, s_tb, lane);
+    }
+    zero_sf_padding(a, s_off, s_tb, warp, lane, kQConsumers / 32);
 }
 
 }  // namespace macaq

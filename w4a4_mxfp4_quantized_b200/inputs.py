@@ -126,18 +126,32 @@ def qwen3_32b_layer(M: int, sweep: int = 0, draw_w: bool = True, device: str = "
 
 @dataclass
 class MoECase:
-    """Grouped linear: X_perm [sum M_e, K] sorted by expert, offsets int32 [E+1], W [E, N, K], s [E, K]."""
+    """Grouped linear: X_perm [sum M_e, K] sorted by expert, offsets int32 [E+1], W [E, N, K], s [E, K].
+    routing: the top-k routing; X_tok: the gate/up input in token order [T, K] (X = X_tok[routing.token]),
+    None for the down projection, whose input is drawn directly in expert-sorted order."""
     name: str
     X: torch.Tensor
     W: torch.Tensor | None
     s: torch.Tensor
     offsets: torch.Tensor
     had_block: int
+    routing: "Routing | None" = None
+    X_tok: torch.Tensor | None = None
 
 
-def moe_routing(g: torch.Generator, T: int, E: int, topk: int, zipf: float = 1.1):
+@dataclass
+class Routing:
+    """Top-k routing of T tokens over E experts, rows sorted by (expert, token)."""
+    token: torch.Tensor     # int64 [T * topk]: the token of each expert-sorted row
+    offsets: torch.Tensor   # int32 [E + 1]: rows of expert e are offsets[e] .. offsets[e+1]
+    pos: torch.Tensor       # int32 [T, topk]: the sorted row of token t's j-th choice
+    weights: torch.Tensor   # fp32 [T, topk]: router weights, softmax over the chosen perturbed scores
+
+
+def moe_routing_full(g: torch.Generator, T: int, E: int, topk: int, zipf: float = 1.1) -> Routing:
     """Zipf(zipf) expert popularity over ranks, mapped to experts by a seeded permutation; each token
-    picks topk distinct experts by Gumbel-top-k on log p. Returns (token index per row, offsets)."""
+    picks topk distinct experts by Gumbel-top-k on log p. The router weights are the softmax of the
+    chosen experts' perturbed scores (no further random draws)."""
     ranks = torch.arange(1, E + 1, dtype=torch.float64)
     p_rank = ranks ** (-zipf)
     p_rank /= p_rank.sum()
@@ -146,14 +160,26 @@ def moe_routing(g: torch.Generator, T: int, E: int, topk: int, zipf: float = 1.1
     logp[perm] = torch.log(p_rank)
     u = torch.rand(T, E, generator=g, dtype=torch.float64).clamp_min(1e-300)
     gumbel = -torch.log(-torch.log(u))
-    choice = torch.topk(logp[None, :] + gumbel, topk, dim=1).indices  # [T, topk]
+    top = torch.topk(logp[None, :] + gumbel, topk, dim=1)
+    choice = top.indices  # [T, topk]
     expert = choice.reshape(-1)
     token = torch.arange(T).repeat_interleave(topk)
     order = torch.argsort(expert * T + token)  # stable by (expert, token)
     counts = torch.bincount(expert, minlength=E)
     offsets = torch.zeros(E + 1, dtype=torch.int32)
     offsets[1:] = torch.cumsum(counts, 0).to(torch.int32)
-    return token[order], offsets
+    inv = torch.empty_like(order)
+    inv[order] = torch.arange(order.numel())
+    pos = inv.reshape(T, topk).to(torch.int32)
+    weights = torch.softmax(top.values, dim=1).to(torch.float32)
+    return Routing(token[order], offsets, pos, weights)
+
+
+def moe_routing(g: torch.Generator, T: int, E: int, topk: int, zipf: float = 1.1):
+    """Zipf(zipf) expert popularity over ranks, mapped to experts by a seeded permutation; each token
+    picks topk distinct experts by Gumbel-top-k on log p. Returns (token index per row, offsets)."""
+    r = moe_routing_full(g, T, E, topk, zipf)
+    return r.token, r.offsets
 
 
 MOE_30B_A3B = dict(E=128, topk=8, hidden=2048, inter=768)
@@ -171,16 +197,18 @@ def moe_30b_a3b(T: int, proj: str = "gate_up", draw_w: bool = True, E: int | Non
     g = _gen(1000 * 4 + 10 * idx + (0 if proj == "gate_up" else 1))
     s = torch.stack([log_uniform_scale(g, K) for _ in range(E)])
     out = outlier_channels(g, K, round(0.005 * K))
-    token, offsets = moe_routing(g, T, E, cfg["topk"])
+    routing = moe_routing_full(g, T, E, cfg["topk"])
+    token, offsets = routing.token, routing.offsets
     sigma = torch.ones(K, dtype=torch.float32)
     sigma[out] *= 30.0
+    X_tok = None
     if proj == "gate_up":
-        Xtok = torch.randn(T, K, generator=g, dtype=torch.float32) * sigma
-        X = Xtok[token].to(torch.bfloat16)
+        X_tok = (torch.randn(T, K, generator=g, dtype=torch.float32) * sigma).to(torch.bfloat16)
+        X = X_tok[token]
     else:
         X = (torch.randn(token.numel(), K, generator=g, dtype=torch.float32) * sigma).to(torch.bfloat16)
     W = normal_bf16(g, (E, N, K), 0.02) if draw_w else None
-    return MoECase(f"moe_30b_a3b_{proj}_T{T}", X, W, s, offsets, 32)
+    return MoECase(f"moe_30b_a3b_{proj}_T{T}", X, W, s, offsets, 32, routing, X_tok)
 
 
 PREFILL_M = (4096, 16384)
