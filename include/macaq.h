@@ -150,6 +150,31 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
                              macaq_stream_t stream);
 
 /*
+ * Flip-Refinement of prepared weights (offline): a coordinate descent over single FP4 codes, guided by
+ * the layer's Hessian, with the E8M0 scales fixed. Per weight row, with w the row's transformed fp32
+ * weights (exactly as macaq_prep_weights computes them from W, s and had_block) and w_hat the codes'
+ * values, it lowers L = (w_hat - w)^T H (w_hat - w):
+ *   g = H (w_hat - w) in float64 (g[i] = sum over k = 0..K-1 in order of H[k][i] (w_hat[k] - w[k]));
+ *   `sweeps` times, for k = 0 .. K-1: try the two neighbouring values on the signed E2M1 grid
+ *   {-6, ..., -0.5, 0, 0.5, ..., 6} at the group's scale, the lower first; a move by d changes L by
+ *   d (2 g[k] + d H[k][k]); the better one (the upper only if strictly better) is taken if that is
+ *   negative, then g[i] += d H[k][i] for all i. Every step is one float64 operation in this order.
+ *   W       device bf16 [N, K] (read), s device fp32 [K] or NULL, had_block as at preparation
+ *   H       device fp32 [K, K], symmetric (e.g. X'^T X' of calibration inputs transformed as for
+ *           macaq_act_quant); row-major
+ *   sweeps  >= 0 (0: no-op)
+ *   Wq      device u8 [N, K/2]: the prepared codes on entry, the refined codes on return
+ *   Wsf     device u8 tiled SF of the N rows from macaq_prep_weights (read, unchanged)
+ *   flips   device int32 [N] (written: accepted moves per row) or NULL; 4-byte aligned
+ *   K % 128 == 0 and K <= 16384 (the per-row state lives in shared memory).
+ * Source: aipolix.com page, paragraph 3 (Flip-Refinement: a Hessian-guided coordinate descent moving
+ * single FP4 codes to neighbouring representable values). The objective and the visiting order are
+ * this library's plain reading; the page gives no formula.
+ */
+macaq_status macaq_flip_refine(const void *W, const float *s, int64_t N, int64_t K, int32_t had_block, const float *H,
+                               int32_t sweeps, uint8_t *Wq, const uint8_t *Wsf, int32_t *flips, macaq_stream_t stream);
+
+/*
  * Activation quantization with a row gather, the dispatch step of a mixture-of-experts layer: output
  * row m is MXFP4( X[row_index[m]] * diag(inv_s) * H_b ), bit-identical to macaq_act_quant applied
  * to the gathered copy X[row_index], which is never written to memory.

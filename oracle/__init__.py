@@ -79,6 +79,8 @@ def _load():
             lib.oracle_swiglu_f32.argtypes = [ctypes.c_float, ctypes.c_float]
             lib.oracle_swiglu_f32.restype = ctypes.c_float
             lib.oracle_swiglu_act_quant.argtypes = [_f32p, _f32p, _f32p, _i64, _i64, ctypes.c_int, _u8p, _u8p, _f32p]
+            lib.oracle_flip_refine.argtypes = [_u16p, _f32p, _i64, _i64, ctypes.c_int, _f32p, ctypes.c_int, _u8p, _u8p,
+                                               _i32p, _f32p, _f64p]
             _lib = lib
     return _lib
 
@@ -324,3 +326,20 @@ def swiglu_act_quant(G, U, inv_s, b: int):
     _load().oracle_swiglu_act_quant(_p(G, _f32p), _p(U, _f32p), _p(inv, _f32p), M, I, int(b), _p(Hq, _u8p),
                                     _p(Hsf, _u8p), _p(work, _f32p))
     return Hq, Hsf
+
+
+def flip_refine(W_bf16, s, b: int, H, sweeps: int, Wq, Wsf):
+    """Flip-Refinement of prepared codes (see macaq_oracle.c): W bf16 [N, K], s [K] or None, H fp32 [K, K]
+    symmetric, Wq [N, K/2] and Wsf [N, K/32] row-major from prep_weights. Returns (refined Wq, flips [N])."""
+    w = _bits16(W_bf16)
+    N, K = w.shape
+    s32 = _f32(s)
+    Hh = np.ascontiguousarray(H, dtype=np.float32)
+    q = np.array(Wq, dtype=np.uint8, copy=True, order="C")
+    sf = np.ascontiguousarray(Wsf, dtype=np.uint8)
+    flips = np.empty(N, np.int32)
+    wrow = np.empty(K, np.float32)
+    g = np.empty(K, np.float64)
+    _load().oracle_flip_refine(_p(w, _u16p), _p(s32, _f32p), N, K, int(b), _p(Hh, _f32p), int(sweeps), _p(q, _u8p),
+                               _p(sf, _u8p), _p(flips, _i32p), _p(wrow, _f32p), _p(g, _f64p))
+    return q, flips

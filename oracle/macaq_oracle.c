@@ -421,3 +421,92 @@ void oracle_swiglu_act_quant(const float *G, const float *U, const float *inv_s,
         oracle_mxfp4_quantize_row(work, I, Hq + m * (I / 2), Hsf + m * (I / MX_GROUP));
     }
 }
+
+/* Signed grid index t in [-7, 7] of an E2M1 code (+0 and -0 are both t = 0), and back. */
+static int e2m1_index(uint8_t code)
+{
+    int m = code & 7;
+    return (code & 8u) ? -m : m;
+}
+
+static uint8_t e2m1_from_index(int t)
+{
+    return t > 0 ? (uint8_t)t : (t < 0 ? (uint8_t)(8 - t) : 0u);
+}
+
+/*
+ * Flip-Refinement of prepared weights. [MACaQ-fa] paragraph 3: a coordinate-descent step, guided by
+ * the Hessian, that moves single FP4 codes to the neighbouring representable values (in place of
+ * GPTQ-style updates). The plain reading taken here, per weight row n:
+ *   w      = the row's transformed fp32 weights, exactly as weight preparation computes them
+ *            (fl32(W s), the fixed-order butterflies per block of b, times 1/b);
+ *   w_hat  = the dequantized codes at the row's E8M0 scales, which never change;
+ *   L      = (w_hat - w)^T H (w_hat - w), H symmetric (e.g. X'^T X' of the layer's transformed
+ *            calibration activations), so L is the squared output error the row's quantization adds.
+ * Keep g = H (w_hat - w) in float64: g[i] = sum over k in order 0..K-1 of H[k][i] * (w_hat[k] - w[k]).
+ * Then `sweeps` times, for k = 0 .. K-1 in order: the candidates are the neighbouring values on the
+ * signed grid {-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, ..., 6} times the group's scale, the lower one
+ * first; moving by d changes L by dL = d * (2 g[k] + d * H[k][k]); the candidate with the smaller dL
+ * (the upper one only if strictly smaller) is taken if dL < 0, and then g[i] += d * H[k][i] for every i.
+ * Every value is exact in float64 (grid values times powers of two); each arithmetic step is one
+ * float64 operation (no multiply-add contraction). A move to zero writes code 0x0.
+ *   W [N, K] bf16 bits, s [K] (NULL: 1), H [K, K] fp32, Wq [N, K/2] (in: the prepared codes; out:
+ *   refined), Wsf [N, K/32] row-major (read), flips [N] (out: accepted moves per row, may be NULL).
+ *   work: K floats (w), K doubles (g).
+ */
+void oracle_flip_refine(const uint16_t *W, const float *s, int64_t N, int64_t K, int b, const float *H, int sweeps,
+                        uint8_t *Wq, const uint8_t *Wsf, int32_t *flips, float *w, double *g)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        uint8_t *q = Wq + n * (K / 2);
+        const uint8_t *sf = Wsf + n * (K / MX_GROUP);
+        oracle_transform_rows(W + n * K, s, 1, K, b, 1, w);
+        for (int64_t i = 0; i < K; ++i)
+            g[i] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t c = (uint8_t)((q[k / 2] >> (4 * (k & 1))) & 15u);
+            double e = ldexp(oracle_e2m1_value(c), (int)sf[k / MX_GROUP] - 127) - (double)w[k];
+            for (int64_t i = 0; i < K; ++i) {
+                double t = (double)H[k * K + i] * e;
+                g[i] = g[i] + t;
+            }
+        }
+        int32_t nflip = 0;
+        for (int sw = 0; sw < sweeps; ++sw) {
+            for (int64_t k = 0; k < K; ++k) {
+                uint8_t c = (uint8_t)((q[k / 2] >> (4 * (k & 1))) & 15u);
+                int t = e2m1_index(c);
+                int E = (int)sf[k / MX_GROUP] - 127;
+                double v = ldexp(oracle_e2m1_value(c), E);
+                double hkk = (double)H[k * K + k];
+                int best_t = t;
+                double best_d = 0.0, best_dl = 0.0;
+                for (int dir = -1; dir <= 1; dir += 2) {
+                    int tc = t + dir;
+                    if (tc < -7 || tc > 7)
+                        continue;
+                    double d = ldexp(oracle_e2m1_value(e2m1_from_index(tc)), E) - v;
+                    double two_g = 2.0 * g[k];
+                    double dh = d * hkk;
+                    double dl = d * (two_g + dh);
+                    if (dl < best_dl) {
+                        best_dl = dl;
+                        best_d = d;
+                        best_t = tc;
+                    }
+                }
+                if (best_t != t) {
+                    uint8_t nc = e2m1_from_index(best_t);
+                    q[k / 2] = (uint8_t)((k & 1) ? ((q[k / 2] & 0x0Fu) | (nc << 4)) : ((q[k / 2] & 0xF0u) | nc));
+                    for (int64_t i = 0; i < K; ++i) {
+                        double t2 = best_d * (double)H[k * K + i];
+                        g[i] = g[i] + t2;
+                    }
+                    ++nflip;
+                }
+            }
+        }
+        if (flips)
+            flips[n] = nflip;
+    }
+}

@@ -463,3 +463,68 @@ def test_swiglu_act_quant_composes_swiglu_transform_and_mxfp4():
         c, s = oracle.swiglu_act_quant(G, U, inv, b)
         np.testing.assert_array_equal(c, c_ref)
         np.testing.assert_array_equal(s, s_ref)
+
+
+# ---------------------------------------------------------------- Flip-Refinement
+def _flip_case(seed, N=6, K=256, b=32, M=512):
+    g = torch.Generator().manual_seed(seed)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    s = torch.exp(torch.rand(K, generator=g) * 2.77 - 0.69).to(torch.float32)
+    X = torch.randn(M, K, generator=g)
+    X[:, :4] *= 20.0                                          # correlated, uneven channels
+    X = (X + 0.5 * X.roll(1, dims=1)).to(torch.bfloat16)
+    Wq, Wsf, inv = oracle.prep_weights(W, s, b)
+    Xt = oracle.transform_rows(X, inv, b, absorb=False).astype(np.float64)
+    H = (Xt.T @ Xt / M).astype(np.float32)
+    w = oracle.transform_rows(W, s, b, absorb=True).astype(np.float64)
+    return W, s, b, Wq, Wsf, H, w
+
+
+def _exact_loss(q, sf, w, H):
+    e = oracle.dequant(q, sf) - w
+    return np.einsum("nk,kj,nj->n", e, H.astype(np.float64), e)
+
+
+def test_flip_refine_separable_hessian_moves_nothing():
+    """With a diagonal positive H the loss separates per code, and the prepared (nearest) codes are
+    already optimal: no move lowers it."""
+    W, s, b, Wq, Wsf, H, w = _flip_case(51)
+    for D in (np.eye(H.shape[0], dtype=np.float32), np.diag(np.diag(H)).astype(np.float32)):
+        q, flips = oracle.flip_refine(W, s, b, D, 2, Wq, Wsf)
+        np.testing.assert_array_equal(q, Wq)
+        assert np.all(flips == 0)
+
+
+def test_flip_refine_loss_never_increases_and_converges_to_a_local_minimum():
+    W, s, b, Wq, Wsf, H, w = _flip_case(52)
+    prev = _exact_loss(Wq, Wsf, w, H)
+    q = Wq
+    total = 0
+    for sweep in range(12):
+        q, flips = oracle.flip_refine(W, s, b, H, 1, q, Wsf)
+        cur = _exact_loss(q, Wsf, w, H)
+        assert np.all(cur <= prev * (1 + 1e-12) + 1e-300), (sweep, cur, prev)
+        total += int(flips.sum())
+        prev = cur
+        if flips.sum() == 0:
+            break
+    assert flips.sum() == 0, "did not converge"
+    assert total > 0 and np.all(prev < _exact_loss(Wq, Wsf, w, H))
+    # brute force: no single neighbouring move lowers the exact loss of any row
+    N, K = w.shape
+    grid = oracle.dequant(q, Wsf)
+    Hd = H.astype(np.float64)
+    E = Wsf.astype(np.int64) - 127
+    vals = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    signed = np.concatenate([-vals[:0:-1], vals])               # index t + 7 for t in [-7, 7]
+    for n in range(N):
+        e = grid[n] - w[n]
+        base = e @ Hd @ e
+        for k in range(K):
+            scale = 2.0 ** E[n, k // 32]
+            t = int(np.argmin(np.abs(signed * scale - grid[n, k])))
+            for tc in (t - 1, t + 1):
+                if 0 <= tc < 15:
+                    e2 = e.copy()
+                    e2[k] += signed[tc] * scale - grid[n, k]
+                    assert e2 @ Hd @ e2 >= base * (1 - 1e-12), (n, k)

@@ -26,7 +26,7 @@ __all__ = [
     "status_str",
     "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
     "set_wait_limit_ns", "check_group_offsets", "act_quant_gather", "moe_combine",
-    "linear_swiglu", "swiglu_act_quant", "interleave_gate_up",
+    "linear_swiglu", "swiglu_act_quant", "interleave_gate_up", "flip_refine",
     "library_path", "lib",
 ]
 
@@ -67,6 +67,7 @@ _SIGNATURES = {
     "macaq_linear_swiglu_workspace_bytes": ([_i64, _i64, _i64], _sz),
     "macaq_linear_swiglu": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "macaq_swiglu_act_quant": ([_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
+    "macaq_flip_refine": ([_vp, _vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
 }
 
 
@@ -266,6 +267,19 @@ def swiglu_act_quant(GU: torch.Tensor, inv_s: torch.Tensor | None, had_block: in
     _check("macaq_swiglu_act_quant", lib().macaq_swiglu_act_quant(
         _ptr(GU), M, I, _ptr(inv_s), had_block, _ptr(Hq), _ptr(Hsf), _stream(dev)))
     return Hq, Hsf
+
+
+def flip_refine(W: torch.Tensor, s: torch.Tensor | None, H: torch.Tensor, Wq: torch.Tensor, Wsf: torch.Tensor,
+                had_block: int = 32, sweeps: int = 1, flips: torch.Tensor | None = None):
+    """Refines the prepared codes Wq in place (Hessian-guided moves to neighbouring FP4 values, scales
+    fixed). H: fp32 CUDA [K, K] symmetric. Returns the per-row count of accepted moves (int32 [N])."""
+    assert W.dtype == torch.bfloat16 and H.dtype == torch.float32
+    N, K = W.shape
+    dev = W.device
+    flips = torch.empty(N, dtype=torch.int32, device=dev) if flips is None else flips
+    _check("macaq_flip_refine", lib().macaq_flip_refine(
+        _ptr(W), _ptr(s), N, K, had_block, _ptr(H), sweeps, _ptr(Wq), _ptr(Wsf), _ptr(flips), _stream(dev)))
+    return flips
 
 
 def _out(M, N, out_dtype, dev, Y):

@@ -16,6 +16,7 @@
 #include <tuple>
 
 #include "macaq.h"
+#include "flip.cuh"
 #include "gemm.cuh"
 #include "moe.cuh"
 #include "quant.cuh"
@@ -804,6 +805,48 @@ macaq_status linear_swiglu(const uint8_t *A, const uint8_t *Asf, int64_t M, int6
     return swiglu_quant(gu, M, I, inv_s, b, hq, hsf, st);
 }
 
+// ------------------------------------------------------------------------ Flip-Refinement
+template <int kCols, int kR>
+macaq_status launch_flip(const FlipArgs &f, int sms, cudaStream_t st) {
+    auto k = flip_refine_kernel<kCols, kR>;
+    const size_t smem = flip_smem_bytes(kR, f.K);
+    macaq_status s = set_smem(k, smem);
+    if (s != MACAQ_OK) return s;
+    const int64_t groups = (static_cast<int64_t>(f.N) + kR - 1) / kR;
+    const unsigned grid = static_cast<unsigned>(groups < sms ? groups : sms);
+    return launch(k, dim3(grid), dim3(kFlipThreads), smem, st, 1, f);
+}
+
+macaq_status flip_refine(const void *W, const float *s, int64_t N, int64_t K, int32_t b, const float *H, int32_t sweeps,
+                         uint8_t *Wq, const uint8_t *Wsf, int32_t *flips, cudaStream_t st) {
+    if (N < 0 || K <= 0 || K % 128 != 0 || K > 16384 || N >= (int64_t(1) << 31) || sweeps < 0) return MACAQ_ERR_SHAPE;
+    if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
+    if (N == 0 || sweeps == 0) return MACAQ_OK;
+    if (W == nullptr || H == nullptr || Wq == nullptr || Wsf == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(s) || !aligned16(H) || !aligned16(Wq) || !aligned16(Wsf) ||
+        (reinterpret_cast<uintptr_t>(flips) & 3u))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status st_ = device_info(&dev);
+    if (st_ != MACAQ_OK) return st_;
+    FlipArgs f;
+    f.w = static_cast<const uint16_t *>(W);
+    f.s = s;
+    f.h = H;
+    f.wq = Wq;
+    f.wsf = Wsf;
+    f.flips = flips;
+    f.N = static_cast<int32_t>(N);
+    f.K = static_cast<int32_t>(K);
+    f.sweeps = sweeps;
+    f.had_block = b;
+    // rows per CTA x columns per thread: 64 float64 sums per thread, shared memory within 227 KB
+    if (K <= 2048) return launch_flip<8, 8>(f, dev.sms, st);
+    if (K <= 4096) return launch_flip<16, 4>(f, dev.sms, st);
+    if (K <= 8192) return launch_flip<32, 2>(f, dev.sms, st);
+    return launch_flip<64, 1>(f, dev.sms, st);
+}
+
 // ------------------------------------------------------------------------ MoE combine
 macaq_status moe_combine(const void *Y, int64_t y_rows, int64_t N, const int32_t *pos, const float *w, int64_t T,
                          int32_t topk, void *out, int32_t out_dtype, cudaStream_t st) {
@@ -925,6 +968,11 @@ macaq_status macaq_linear_swiglu(const uint8_t *A, const uint8_t *Asf, int64_t M
 macaq_status macaq_swiglu_act_quant(const float *GU, int64_t M, int64_t I, const float *inv_s, int32_t had_block,
                                     uint8_t *Hq, uint8_t *Hsf, macaq_stream_t stream) {
     return macaq::swiglu_quant(GU, M, I, inv_s, had_block, Hq, Hsf, static_cast<cudaStream_t>(stream));
+}
+
+macaq_status macaq_flip_refine(const void *W, const float *s, int64_t N, int64_t K, int32_t had_block, const float *H,
+                               int32_t sweeps, uint8_t *Wq, const uint8_t *Wsf, int32_t *flips, macaq_stream_t stream) {
+    return macaq::flip_refine(W, s, N, K, had_block, H, sweeps, Wq, Wsf, flips, static_cast<cudaStream_t>(stream));
 }
 
 macaq_status macaq_moe_combine(const void *Y, int64_t y_rows, int64_t N, const int32_t *pos, const float *weights,
