@@ -335,6 +335,21 @@ def moe_section(dev, hbm, fp4_peak, steps=20):
             aq = time_graph(lambda i: mq.act_quant(Xs[i % 2], inv, HAD_BLOCK, group_offsets=off, Xq=Xq[i % 2],
                                                    Xsf=Xsf[i % 2]), steps, stream)
             gm = time_graph(lambda i: mq.grouped_linear(Xq[i % 2], Xsf[i % 2], off, Wq, Wsf, Y=Y), steps, stream)
+            glue = {}
+            if proj == "gate_up":   # dispatch: quantize token rows through the routing's row index
+                Xt = [c.X_tok.to(dev), c.X_tok.to(dev).clone()]
+                idx = c.routing.token.to(torch.int32).to(dev)
+                glue["gather_act_quant_us"] = 1e3 * time_graph(
+                    lambda i: mq.act_quant_gather(Xt[i % 2], idx, inv, HAD_BLOCK, group_offsets=off, Xq=Xq[i % 2],
+                                                  Xsf=Xsf[i % 2]), steps, stream)
+                del Xt
+            else:                   # combine: the down projection's rows back to token order, weighted
+                pos, wts = c.routing.pos.to(dev), c.routing.weights.to(dev)
+                out_t = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+                cm = time_graph(lambda i: mq.moe_combine(Y, pos, wts, out=out_t), steps, stream)
+                c_bytes = rows * N * 2 + T * N * 2 + T * 8 * 8
+                glue.update({"combine_us": cm * 1e3, "combine_gbs": c_bytes / (cm * 1e-3) / 1e9,
+                             "combine_frac_hbm": c_bytes / (cm * 1e-3) / 1e9 / hbm})
             assert mq.device_status() == 0
             flops = 2.0 * N * K * rows
             used = int((counts > 0).sum())
@@ -346,7 +361,7 @@ def moe_section(dev, hbm, fp4_peak, steps=20):
                         "grouped_gemm_frac_fp4_peak": flops / (gm * 1e-3) / 1e12 / fp4_peak,
                         "grouped_gemm_frac_hbm": g_bytes / (gm * 1e-3) / 1e9 / hbm,
                         "grouped_act_quant_us": aq * 1e3, "grouped_act_quant_gbs": a_bytes / (aq * 1e-3) / 1e9,
-                        "grouped_act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm})
+                        "grouped_act_quant_frac_hbm": a_bytes / (aq * 1e-3) / 1e9 / hbm, **glue})
             del Xs, Xq, Xsf, Y
         del Wq, Wsf, inv
     return {"workload": f"moe_30b_a3b E=128 top-8, gate/up 2048->1536 and down 768->2048, b={HAD_BLOCK}",
@@ -538,6 +553,42 @@ def copy_ceiling(dev, nbytes, steps=20):
     return {"bytes": int(nbytes), "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9}
 
 
+def flip_section(dev, sweeps=1):
+    """Flip-Refinement of the Llama-3-8B up/gate weights [14336, 4096] with a Hessian from 512
+    transformed calibration rows (the Hessian product is plumbing: torch, fp32). One timed call."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    c = inputs.llama3_8b_up(2048)
+    W, s = c.W.to(dev), c.s.to(dev)
+    Wq, Wsf, inv = mq.prep_weights(W, s, HAD_BLOCK)
+    Xt = (c.X[:512].to(dev).float() * inv)
+    Xt = Xt.view(512, -1, HAD_BLOCK) @ torch.from_numpy(_sylvester(HAD_BLOCK)).to(dev)
+    Xt = Xt.view(512, -1)
+    H = (Xt.T @ Xt / 512).contiguous()
+    q = Wq.clone()
+    mq.flip_refine(W, s, H, q, Wsf, HAD_BLOCK, sweeps)          # warm-up (and the module load)
+    torch.cuda.synchronize()
+    q.copy_(Wq)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(dev)
+    a.record(stream)
+    flips = mq.flip_refine(W, s, H, q, Wsf, HAD_BLOCK, sweeps)
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert mq.device_status() == 0
+    return {"workload": f"llama3_8b_up_gate W [{N_DIM}, {K_DIM}], H from 512 rows, {sweeps} sweep(s)",
+            "ms": a.elapsed_time(b), "moves_per_row": float(flips.float().mean()),
+            "codes_changed_frac": float((q != Wq).float().mean())}
+
+
+def _sylvester(b):
+    h = np.ones((1, 1), np.float32)
+    while h.shape[0] < b:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
 def weight_prep_section(dev, hbm, steps=10):
     """Offline weight preparation of the Llama-3-8B up/gate weights (bf16 in, codes + SF out)."""
     import w4a4_mxfp4_quantized_b200 as mq
@@ -667,7 +718,7 @@ def _r(x, n=3):
     return None if x is None else float(f"{x:.{n}g}")
 
 
-def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling):
+def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None):
     """Short strings of the sections, so that the whole line stays a few KB."""
     out = {}
     if sweep:
@@ -688,9 +739,18 @@ def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling):
             f"swiglu chain {p['layer_swiglu_chain_us']:.0f}us (gate/up+swiglu {p['swiglu_fused_us']:.0f} vs "
             f"{p['swiglu_two_step_us']:.0f}us)" for p in qwen3["points"])
     if moe:
+        def glue(p):
+            if "gather_act_quant_us" in p:
+                return f", gather aq {p['gather_act_quant_us']:.1f}us vs {p['grouped_act_quant_us']:.1f}"
+            if "combine_us" in p:
+                return f", combine {p['combine_us']:.1f}us {p['combine_frac_hbm']:.2f}hbm"
+            return ""
         out["moe"] = " | ".join(
             f"{p['proj']} T{p['T']}: gemm {p['grouped_gemm_us']:.1f}us {p['grouped_gemm_frac_hbm']:.2f}hbm "
-            f"{p['grouped_gemm_frac_fp4_peak']:.2f}fp4, aq {p['grouped_act_quant_frac_hbm']:.2f}hbm" for p in moe["points"])
+            f"{p['grouped_gemm_frac_fp4_peak']:.2f}fp4, aq {p['grouped_act_quant_frac_hbm']:.2f}hbm{glue(p)}"
+            for p in moe["points"])
+    if flip:
+        out["flip_refine"] = f"{flip['ms']:.1f}ms, {flip['moves_per_row']:.0f} moves/row"
     if prep:
         out["weight_prep"] = f"{prep['us']:.1f}us {prep['frac_hbm']:.2f}hbm"
     if ceiling:
@@ -747,7 +807,7 @@ def main():
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     gemm_kernel = gemm_kernel_name(M)
     aq_bytes = M * K_DIM * (2 + 0.5 + 1 / 32)
-    sweep, prefill, qwen3, moe, prep, ceiling = [], None, None, None, None, []
+    sweep, prefill, qwen3, moe, prep, ceiling, flip = [], None, None, None, None, [], None
     if not args.no_sweep:
         for m in M_SWEEP:
             tot, aq, gm, Lm = time_layer(m, max(10, args.steps), args.warmup, dev, dist_on, fused=True)
@@ -771,6 +831,7 @@ def main():
         qwen3 = qwen3_section(dev, hbm, fp4_peak)
         moe = moe_section(dev, hbm, fp4_peak)
         prep = weight_prep_section(dev, hbm)
+        flip = flip_section(dev)
         ceiling = [copy_ceiling(dev, aq_bytes), copy_ceiling(dev, 16384 * 16384 * 2.53125)]
     if rank != 0:
         if dist_on:
@@ -796,11 +857,11 @@ def main():
         "clocks": dict(clocks, window="warm replays (1.5 s of this workload) and the timed replay"),
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
-    out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling)
+    out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip)
     if args.details:
         with open(args.details, "w") as f:
             json.dump({**out, "sweep": sweep, "transform_overhead": overhead, "prefill": prefill, "qwen3": qwen3,
-                       "moe": moe, "weight_prep": prep, "copy_ceiling": ceiling}, f, indent=1)
+                       "moe": moe, "weight_prep": prep, "copy_ceiling": ceiling, "flip_refine": flip}, f, indent=1)
     print(json.dumps(out))
     if dist_on:
         torch.distributed.destroy_process_group()

@@ -150,6 +150,36 @@ macaq_status macaq_act_quant(const void *X, const float *inv_s, int64_t M, int64
                              macaq_stream_t stream);
 
 /*
+ * The weight-only mode's activation transform: Xt = bf16( X * diag(inv_s) * H_b ), the act_quant
+ * arithmetic (fp32 multiply, fixed-order butterflies) with each value rounded once to bf16 (nearest
+ * even) instead of MXFP4.
+ *   X device bf16 [M, K] (read); inv_s device fp32 [K] or NULL; had_block b; Xt device bf16 [M, K]
+ *   (written). K % 128 == 0.
+ * Sources: glonce.com page, paragraph 3 (vLLM serves W4A4 or weight-only checkpoints); aipolix.com
+ * page, paragraph 2 (the transform at the input of every linear).
+ */
+macaq_status macaq_act_transform(const void *X, const float *inv_s, int64_t M, int64_t K, int32_t had_block, void *Xt,
+                                 macaq_stream_t stream);
+
+/*
+ * Weight-only (W4A16) linear for decode and small batches:
+ *     Y[m, n] = sum_k bf16(X'[m, k]) * dq(W'[n, k]),  X' = X * diag(inv_s) * H_b (macaq_act_transform)
+ * with the weights prepared by macaq_prep_weights exactly as for W4A4 (codes + tiled SF) and fp32
+ * accumulation on the tensor cores (kind::f16, bf16 x bf16): the weight codes are expanded to bf16
+ * inside the kernel (exact for scales E8M0 <= 252) and never written to memory.
+ *   X           device bf16 [M, K], 1 <= M <= 128 (M == 0 is a no-op); K % 256 == 0; N % 128 == 0
+ *   inv_s, had_block  as for macaq_act_quant; Wq, Wsf as for macaq_linear
+ *   Y           device [M, N], bf16 or fp32 per out_dtype (written)
+ *   workspace   at least macaq_linear_w4a16_workspace_bytes(M, N, K) bytes (the transformed
+ *               activations and the split-tile scratch), under the contract of macaq_workspace_bytes
+ * Source: glonce.com page, paragraph 3 (weight-only mode).
+ */
+size_t macaq_linear_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+macaq_status macaq_linear_w4a16(const void *X, const float *inv_s, int64_t M, int64_t N, int64_t K, int32_t had_block,
+                                const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
+                                size_t ws_bytes, macaq_stream_t stream);
+
+/*
  * Flip-Refinement of prepared weights (offline): a coordinate descent over single FP4 codes, guided by
  * the layer's Hessian, with the E8M0 scales fixed. Per weight row, with w the row's transformed fp32
  * weights (exactly as macaq_prep_weights computes them from W, s and had_block) and w_hat the codes'

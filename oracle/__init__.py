@@ -79,6 +79,7 @@ def _load():
             lib.oracle_swiglu_f32.argtypes = [ctypes.c_float, ctypes.c_float]
             lib.oracle_swiglu_f32.restype = ctypes.c_float
             lib.oracle_swiglu_act_quant.argtypes = [_f32p, _f32p, _f32p, _i64, _i64, ctypes.c_int, _u8p, _u8p, _f32p]
+            lib.oracle_act_transform_bf16.argtypes = [_u16p, _f32p, _i64, _i64, ctypes.c_int, _u16p, _f32p]
             lib.oracle_flip_refine.argtypes = [_u16p, _f32p, _i64, _i64, ctypes.c_int, _f32p, ctypes.c_int, _u8p, _u8p,
                                                _i32p, _f32p, _f64p]
             _lib = lib
@@ -343,3 +344,39 @@ def flip_refine(W_bf16, s, b: int, H, sweeps: int, Wq, Wsf):
     _load().oracle_flip_refine(_p(w, _u16p), _p(s32, _f32p), N, K, int(b), _p(Hh, _f32p), int(sweeps), _p(q, _u8p),
                                _p(sf, _u8p), _p(flips, _i32p), _p(wrow, _f32p), _p(g, _f64p))
     return q, flips
+
+
+def act_transform_bf16(X_bf16, inv_s, b: int) -> np.ndarray:
+    """bf16 bits [M, K] of X diag(inv_s) H_b computed in fp32 and rounded once (weight-only activations)."""
+    x = _bits16(X_bf16)
+    M, K = x.shape
+    inv = _f32(inv_s)
+    out = np.empty((M, K), np.uint16)
+    work = np.empty(K, np.float32)
+    _load().oracle_act_transform_bf16(_p(x, _u16p), _p(inv, _f32p), M, K, int(b), _p(out, _u16p), _p(work, _f32p))
+    return out
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact float64 values of bf16 bit patterns."""
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def w4a16_linear(X_bf16, inv_s, b: int, Wq, Wsf, rows=None, n_chunk: int = 4096):
+    """The weight-only layer: Y = bf16(X diag(inv_s) H_b) dq(W')^T and T = |.| |.|^T in float64 (the k-sum by a
+    library matmul, as linear_matmul), for the listed rows of X."""
+    xt = act_transform_bf16(X_bf16 if rows is None else _rows16(X_bf16, rows), inv_s, b)
+    a = bf16_bits_to_f64(xt)
+    a_abs = np.abs(a)
+    N = Wq.shape[0]
+    Y = np.empty((a.shape[0], N), np.float64)
+    T = np.empty((a.shape[0], N), np.float64)
+    for n0 in range(0, N, n_chunk):
+        w = dequant(np.ascontiguousarray(Wq[n0:n0 + n_chunk]), np.ascontiguousarray(Wsf[n0:n0 + n_chunk]))
+        Y[:, n0:n0 + w.shape[0]] = a @ w.T
+        T[:, n0:n0 + w.shape[0]] = a_abs @ np.abs(w).T
+    return Y, T
+
+
+def _rows16(X_bf16, rows):
+    return np.ascontiguousarray(_bits16(X_bf16)[np.asarray(rows, dtype=np.int64)])

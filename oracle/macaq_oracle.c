@@ -510,3 +510,19 @@ void oracle_flip_refine(const uint16_t *W, const float *s, int64_t N, int64_t K,
             flips[n] = nflip;
     }
 }
+
+/*
+ * The weight-only mode's activations: X * diag(1/s) * H_b in fp32 (the act_quant transform), each value
+ * then rounded once to bf16 (nearest even). [MACaQ-en] paragraph 3 (vLLM serves W4A4 or weight-only
+ * checkpoints); [MACaQ-fa] paragraph 2 (the transform at the input of every linear).
+ *   X [M, K] bf16 bits, inv_s [K] (NULL: 1) -> Xt [M, K] bf16 bits. work: K floats.
+ */
+void oracle_act_transform_bf16(const uint16_t *X, const float *inv_s, int64_t M, int64_t K, int b, uint16_t *Xt,
+                               float *work)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        oracle_transform_rows(X + m * K, inv_s, 1, K, b, 0, work);
+        for (int64_t k = 0; k < K; ++k)
+            Xt[m * K + k] = oracle_bf16_rne(work[k]);
+    }
+}

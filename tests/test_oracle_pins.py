@@ -528,3 +528,56 @@ def test_flip_refine_loss_never_increases_and_converges_to_a_local_minimum():
                     e2 = e.copy()
                     e2[k] += signed[tc] * scale - grid[n, k]
                     assert e2 @ Hd @ e2 >= base * (1 - 1e-12), (n, k)
+
+
+# ---------------------------------------------------------------- weight-only (W4A16)
+def test_act_transform_bf16_composes_transform_and_rounding():
+    g = torch.Generator().manual_seed(61)
+    X = (torch.randn(7, 512, generator=g) * 10).to(torch.bfloat16)
+    inv = (1.0 / torch.exp(torch.rand(512, generator=g) * 2.77 - 0.69)).to(torch.float32).numpy()
+    for b in (1, 16, 32, 64, 128):
+        ref = torch.from_numpy(oracle.transform_rows(X, inv, b, absorb=False)).to(torch.bfloat16)
+        got = oracle.act_transform_bf16(X, inv, b)
+        np.testing.assert_array_equal(got, ref.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_w4a16_linear_exact_on_tiny_inputs():
+    """b = 1 and no s: the activations are X itself (already bf16), so Y is the exact rational sum of
+    X times the dequantized codes."""
+    rng = np.random.default_rng(62)
+    M, N, K = 3, 4, 64
+    X = torch.from_numpy(rng.normal(0, 1, (M, K)).astype(np.float32)).to(torch.bfloat16)
+    Wq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    Wsf = rng.integers(110, 140, (N, K // 32), dtype=np.uint8)
+    Y, T = oracle.w4a16_linear(X, None, 1, Wq, Wsf)
+    xv = [[Fraction(float(v)) for v in row] for row in X.float().numpy()]
+    for m in range(M):
+        for n in range(N):
+            terms = []
+            for k in range(K):
+                c = (Wq[n, k // 2] >> (4 * (k & 1))) & 15
+                w = (-1 if c & 8 else 1) * Fraction(GRID[c & 7]) * Fraction(2) ** (int(Wsf[n, k // 32]) - 127)
+                terms.append(xv[m][k] * w)
+            tabs = sum((abs(t) for t in terms), Fraction(0))
+            assert abs(Fraction(Y[m, n]) - sum(terms, Fraction(0))) <= Fraction(1, 10 ** 12) * tabs
+            assert abs(Fraction(T[m, n]) - tabs) <= Fraction(1, 10 ** 12) * tabs
+
+
+def test_w4a16_beats_w4a4_on_outlier_channels():
+    """With outlier channels, keeping the (transformed) activations in bf16 loses less than MXFP4
+    activations: the weight-only layer is closer to X W^T than the W4A4 layer."""
+    g = torch.Generator().manual_seed(63)
+    M, K, N, b = 16, 1024, 64, 32
+    X = torch.randn(M, K, generator=g)
+    X[:, [5, 300, 777]] *= 40
+    X = X.to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    s = torch.exp(torch.rand(K, generator=g) * 2.77 - 0.69).to(torch.float32)
+    ref = X.double().numpy() @ W.double().numpy().T
+    Wq, Wsf, inv = oracle.prep_weights(W, s, b)
+    Yw, _ = oracle.w4a16_linear(X, inv, b, Wq, Wsf)
+    Xq, Xsf = oracle.act_quant(X, inv, b)
+    Ya, _ = oracle.linear(Xq, Xsf, Wq, Wsf)
+    err_w = np.linalg.norm(Yw - ref) / np.linalg.norm(ref)
+    err_a = np.linalg.norm(Ya - ref) / np.linalg.norm(ref)
+    assert err_w < err_a, (err_w, err_a)

@@ -26,7 +26,7 @@ __all__ = [
     "status_str",
     "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
     "set_wait_limit_ns", "check_group_offsets", "act_quant_gather", "moe_combine",
-    "linear_swiglu", "swiglu_act_quant", "interleave_gate_up", "flip_refine",
+    "linear_swiglu", "swiglu_act_quant", "interleave_gate_up", "flip_refine", "act_transform", "linear_w4a16",
     "library_path", "lib",
 ]
 
@@ -68,6 +68,9 @@ _SIGNATURES = {
     "macaq_linear_swiglu": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "macaq_swiglu_act_quant": ([_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
     "macaq_flip_refine": ([_vp, _vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "macaq_act_transform": ([_vp, _vp, _i64, _i64, _i32, _vp, _vp], ctypes.c_int),
+    "macaq_linear_w4a16_workspace_bytes": ([_i64, _i64, _i64], _sz),
+    "macaq_linear_w4a16": ([_vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _i32, _vp, _sz, _vp], ctypes.c_int),
 }
 
 
@@ -280,6 +283,34 @@ def flip_refine(W: torch.Tensor, s: torch.Tensor | None, H: torch.Tensor, Wq: to
     _check("macaq_flip_refine", lib().macaq_flip_refine(
         _ptr(W), _ptr(s), N, K, had_block, _ptr(H), sweeps, _ptr(Wq), _ptr(Wsf), _ptr(flips), _stream(dev)))
     return flips
+
+
+def act_transform(X: torch.Tensor, inv_s: torch.Tensor | None, had_block: int = 32, *, Xt=None):
+    """bf16(X diag(inv_s) H_b): the weight-only mode's activations (the act_quant transform, no MXFP4)."""
+    assert X.dtype == torch.bfloat16 and X.dim() == 2
+    M, K = X.shape
+    Xt = torch.empty(M, K, dtype=torch.bfloat16, device=X.device) if Xt is None else Xt
+    _check("macaq_act_transform", lib().macaq_act_transform(_ptr(X), _ptr(inv_s), M, K, had_block, _ptr(Xt),
+                                                            _stream(X.device)))
+    return Xt
+
+
+def linear_w4a16(X: torch.Tensor, inv_s: torch.Tensor | None, Wq: torch.Tensor, Wsf: torch.Tensor, *,
+                 had_block: int = 32, out_dtype: int = OUT_BF16, Y=None, workspace=None):
+    """Weight-only layer for decode (M <= 128): Y = bf16(X diag(inv_s) H_b) dq(W')^T, fp32 accumulation."""
+    N = Wq.shape[0]
+    K = Wq.shape[1] * 2
+    M = X.shape[0]
+    dev = X.device
+    Y = _out(M, N, out_dtype, dev, Y)
+    need = int(lib().macaq_linear_w4a16_workspace_bytes(M, N, K))
+    if workspace is None and need > 0:
+        workspace = _workspace(dev, need)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("macaq_linear_w4a16", lib().macaq_linear_w4a16(
+        _ptr(X), _ptr(inv_s), M, N, K, had_block, _ptr(Wq), _ptr(Wsf), _ptr(Y), out_dtype, _ptr(workspace), ws_bytes,
+        _stream(dev)))
+    return Y
 
 
 def _out(M, N, out_dtype, dev, Y):

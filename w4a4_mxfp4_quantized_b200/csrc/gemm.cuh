@@ -711,6 +711,127 @@ __host__ __device__ constexpr int skinny_stage_bytes(int mp) { return 128 * kBKB
 __host__ __device__ constexpr int skinny_stage_bytes_fused(int mp) { return skinny_stage_bytes(mp) + mp * 512 + 1024; }
 __host__ __device__ constexpr int skinny_stage_bytes_y(int mp) { return mp * 128 * 2; }  // bf16 staging of one tile
 
+// Epilogue of the skinny kernels (warps 2-5, one TMEM lane quarter each): for every piece of a weight
+// tile this CTA covers, wait for its accumulator (buffer b = piece parity at tmem + 128 b), then either
+// write Y (a tile covered by one CTA: bf16 staged in shared memory and stored by TMA, or fp32 direct)
+// or publish the piece's fp32 partial and, in the CTA that completes the tile, add the pieces in their
+// fixed order and write Y. The CTA covering unit u is the largest c with floor(c * chunks / C) <= u /
+// gran, C = gridDim.x.
+__device__ __forceinline__ void skinny_epilogue(const SkinnyArgs &g, const CUtensorMap *ymap, uint32_t tmem, int warp, int lane,
+                                                uint8_t *sY, int mp, uint64_t *accum_full, uint64_t *accum_empty,
+                                                volatile int *failed, int32_t *s_last, uint64_t limit, uint32_t u_begin,
+                                                uint32_t u_end, uint32_t num_kb, uint32_t chunks) {
+    const uint32_t C = gridDim.x;
+    auto cta_of = [&](uint32_t u) {
+        return static_cast<uint32_t>(((static_cast<uint64_t>(u / g.gran) + 1) * C - 1) / chunks);
+    };
+    const int quarter = warp & 3;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int nl = quarter * 32 + lane;          // W row inside the tile
+    uint8_t *ystage = sY + static_cast<size_t>(quarter) * mp * 64;  // [mp][32] bf16 of this warp
+    uint32_t piece = 0;
+    for (uint32_t u = u_begin; u < u_end; ++piece) {
+        const uint32_t tile = u / num_kb;
+        const uint32_t u_first = tile * num_kb;
+        const uint32_t u_stop = min(u_end, u_first + num_kb);
+        const uint32_t c_first = cta_of(u_first), c_last = cta_of(u_first + num_kb - 1);
+        const int npieces = static_cast<int>(c_last - c_first + 1);
+        const int pidx = static_cast<int>(blockIdx.x - c_first);
+        u = u_stop;
+        const int b = piece & 1;
+        bool ok = mbar_wait_or_abort(&accum_full[b], (piece >> 1) & 1, limit, failed);
+        tc_fence_after();
+        // the four epilogue warps meet at named barriers below (split tiles): they stop together
+        // or not at all, so a wait that ran out in one warp never leaves the others at a barrier
+        if (!bar_and(1, 128, ok && !*failed)) break;
+        const int64_t n = static_cast<int64_t>(tile) * 128 + nl;
+        const bool staged = npieces == 1 && !g.out_f32;
+        if (staged) {  // the previous tile's store (issued by lane 0) has read the staging buffer
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+        }
+        float *part = g.partials + ((static_cast<uint64_t>(tile) * g.max_pieces + pidx) * g.M) * 128;
+        auto emit = [&](int m0, const uint32_t (&v)[32]) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int m = m0 + i;
+                const float f = __uint_as_float(v[i]);
+                if (staged) {
+                    if (m < mp) reinterpret_cast<__nv_bfloat16 *>(ystage)[m * 32 + lane] = __float2bfloat16_rn(f);
+                } else if (m < g.M) {
+                    if (npieces == 1) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = f;
+                    else __stcg(part + static_cast<int64_t>(m) * 128 + nl, f);
+                }
+            }
+        };
+        for (int m0 = 0; m0 < mp; m0 += 64) {  // two TMEM loads in flight per wait
+            uint32_t v0[32], v1[32];
+            tmem_ld32(taddr + 128 * b + m0, v0);
+            if (m0 + 32 < mp) tmem_ld32(taddr + 128 * b + m0 + 32, v1);
+            tmem_ld_wait();
+            emit(m0, v0);
+            if (m0 + 32 < mp) emit(m0 + 32, v1);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accum_empty[b]);
+        if (staged) {
+            fence_proxy_async_smem();  // generic writes -> the TMA store's reads
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(ymap, ystage, static_cast<int32_t>(tile * 128 + quarter * 32), 0);
+                bulk_commit();
+            }
+        }
+        if (npieces > 1) {
+            // publish this piece, then let the CTA that completes the tile add the pieces in order.
+            // The barrier orders every thread's partial stores before thread 0's fence and count
+            // increment (a cumulative release); the reader side mirrors it.
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (warp == 2 && lane == 0) {
+                __threadfence();
+                *s_last = atomicAdd(&g.counts[tile], 1) == npieces - 1;
+                __threadfence();
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (*s_last) {
+                // the pieces are added in their fixed order (piece 0 first); four pieces x 16 rows of
+                // loads are in flight per round trip to L2
+                float *base = g.partials + (static_cast<uint64_t>(tile) * g.max_pieces) * g.M * 128 + nl;
+                for (int m0 = 0; m0 < g.M; m0 += 16) {
+                    float acc[16];
+                    for (int p0 = 0; p0 < npieces; p0 += 4) {
+                        float v[4][16];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                v[q][i] = (p0 + q < npieces && m0 + i < g.M)
+                                              ? __ldcg(base + (static_cast<uint64_t>(p0 + q) * g.M + m0 + i) * 128)
+                                              : 0.0f;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (p0 + q >= npieces) break;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) acc[i] = (p0 + q == 0) ? v[q][i] : acc[i] + v[q][i];
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int m = m0 + i;
+                        if (m >= g.M) break;
+                        if (g.out_f32) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = acc[i];
+                        else static_cast<__nv_bfloat16 *>(g.y)[static_cast<int64_t>(m) * g.N + n] = __float2bfloat16_rn(acc[i]);
+                    }
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (warp == 2 && lane == 0) g.counts[tile] = 0;  // ready for the next call
+            }
+        }
+    }
+    if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it
+}
+
 template <int kFusedB>
 __global__ void __launch_bounds__(kFusedB > 0 ? 320 : 192, 1)
 gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
@@ -750,10 +871,6 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
     const uint32_t u_begin = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x) * chunks) / C) * g.gran;
     const uint32_t u_end = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x + 1) * chunks) / C) * g.gran;
     const uint64_t limit = g.wait_limit_ns;
-    // CTA covering unit u (the ranges above): largest c with floor(c * chunks / C) <= u / gran
-    auto cta_of = [&](uint32_t u) {
-        return static_cast<uint32_t>(((static_cast<uint64_t>(u / g.gran) + 1) * C - 1) / chunks);
-    };
 
     // The weights do not depend on the previous kernel in the stream, and their loads need only this
     // CTA's barriers: thread 0 requests the first stages' W' tiles and scale factors right after it
@@ -930,111 +1047,8 @@ gemm_mxf4_skinny_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_c
         }
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2-5)
-        const int quarter = warp & 3;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        const int nl = quarter * 32 + lane;          // W row inside the tile
-        uint8_t *ystage = sY + static_cast<size_t>(quarter) * mp * 64;  // [mp][32] bf16 of this warp
-        uint32_t piece = 0;
-        for (uint32_t u = u_begin; u < u_end; ++piece) {
-            const uint32_t tile = u / num_kb;
-            const uint32_t u_first = tile * num_kb;
-            const uint32_t u_stop = min(u_end, u_first + num_kb);
-            const uint32_t c_first = cta_of(u_first), c_last = cta_of(u_first + num_kb - 1);
-            const int npieces = static_cast<int>(c_last - c_first + 1);
-            const int pidx = static_cast<int>(blockIdx.x - c_first);
-            u = u_stop;
-            const int b = piece & 1;
-            bool ok = mbar_wait_or_abort(&accum_full[b], (piece >> 1) & 1, limit, &failed);
-            tc_fence_after();
-            // the four epilogue warps meet at named barriers below (split tiles): they stop together
-            // or not at all, so a wait that ran out in one warp never leaves the others at a barrier
-            if (!bar_and(1, 128, ok && !failed)) break;
-            const int64_t n = static_cast<int64_t>(tile) * 128 + nl;
-            const bool staged = npieces == 1 && !g.out_f32;
-            if (staged) {  // the previous tile's store (issued by lane 0) has read the staging buffer
-                if (lane == 0) bulk_wait_read();
-                __syncwarp();
-            }
-            float *part = g.partials + ((static_cast<uint64_t>(tile) * g.max_pieces + pidx) * g.M) * 128;
-            auto emit = [&](int m0, const uint32_t (&v)[32]) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int m = m0 + i;
-                    const float f = __uint_as_float(v[i]);
-                    if (staged) {
-                        if (m < mp) reinterpret_cast<__nv_bfloat16 *>(ystage)[m * 32 + lane] = __float2bfloat16_rn(f);
-                    } else if (m < g.M) {
-                        if (npieces == 1) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = f;
-                        else __stcg(part + static_cast<int64_t>(m) * 128 + nl, f);
-                    }
-                }
-            };
-            for (int m0 = 0; m0 < mp; m0 += 64) {  // two TMEM loads in flight per wait
-                uint32_t v0[32], v1[32];
-                tmem_ld32(taddr + 128 * b + m0, v0);
-                if (m0 + 32 < mp) tmem_ld32(taddr + 128 * b + m0 + 32, v1);
-                tmem_ld_wait();
-                emit(m0, v0);
-                if (m0 + 32 < mp) emit(m0 + 32, v1);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&accum_empty[b]);
-            if (staged) {
-                fence_proxy_async_smem();  // generic writes -> the TMA store's reads
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&ymap, ystage, static_cast<int32_t>(tile * 128 + quarter * 32), 0);
-                    bulk_commit();
-                }
-            }
-            if (npieces > 1) {
-                // publish this piece, then let the CTA that completes the tile add the pieces in order.
-                // The barrier orders every thread's partial stores before thread 0's fence and count
-                // increment (a cumulative release); the reader side mirrors it.
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (warp == 2 && lane == 0) {
-                    __threadfence();
-                    s_last = atomicAdd(&g.counts[tile], 1) == npieces - 1;
-                    __threadfence();
-                }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (s_last) {
-                    // the pieces are added in their fixed order (piece 0 first); four pieces x 16 rows of
-                    // loads are in flight per round trip to L2
-                    float *base = g.partials + (static_cast<uint64_t>(tile) * g.max_pieces) * g.M * 128 + nl;
-                    for (int m0 = 0; m0 < g.M; m0 += 16) {
-                        float acc[16];
-                        for (int p0 = 0; p0 < npieces; p0 += 4) {
-                            float v[4][16];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                                for (int i = 0; i < 16; ++i)
-                                    v[q][i] = (p0 + q < npieces && m0 + i < g.M)
-                                                  ? __ldcg(base + (static_cast<uint64_t>(p0 + q) * g.M + m0 + i) * 128)
-                                                  : 0.0f;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                if (p0 + q >= npieces) break;
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) acc[i] = (p0 + q == 0) ? v[q][i] : acc[i] + v[q][i];
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int m = m0 + i;
-                            if (m >= g.M) break;
-                            if (g.out_f32) static_cast<float *>(g.y)[static_cast<int64_t>(m) * g.N + n] = acc[i];
-                            else static_cast<__nv_bfloat16 *>(g.y)[static_cast<int64_t>(m) * g.N + n] = __float2bfloat16_rn(acc[i]);
-                        }
-                    }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    if (warp == 2 && lane == 0) g.counts[tile] = 0;  // ready for the next call
-                }
-            }
-        }
-        if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it
+        skinny_epilogue(g, &ymap, tmem, warp, lane, sY, mp, accum_full, accum_empty, &failed, &s_last, limit, u_begin,
+                        u_end, num_kb, chunks);
     }
 
     tc_fence_before();

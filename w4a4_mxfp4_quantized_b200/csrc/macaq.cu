@@ -20,6 +20,7 @@
 #include "gemm.cuh"
 #include "moe.cuh"
 #include "quant.cuh"
+#include "w4a16.cuh"
 
 namespace macaq {
 
@@ -186,23 +187,23 @@ macaq_status launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStrea
 }
 
 // ------------------------------------------------------------------------ quantization
-template <int kB, bool kWeight>
+template <int kB, bool kWeight, bool kBf16Out = false>
 macaq_status run_quant_b(const CUtensorMap &map, const QuantArgs &a, int grid, cudaStream_t st) {
-    auto k = quant_kernel<kB, kWeight>;
+    auto k = quant_kernel<kB, kWeight, kBf16Out>;
     const size_t smem = quant_smem_bytes(a.E);
     macaq_status s = set_smem(k, smem);
     if (s != MACAQ_OK) return s;
     return launch(k, dim3(grid), dim3(kQThreads), smem, st, 1, map, a);
 }
 
-template <bool kWeight>
+template <bool kWeight, bool kBf16Out = false>
 macaq_status run_quant(int32_t b, const CUtensorMap &map, const QuantArgs &a, int grid, cudaStream_t st) {
     switch (b) {
-        case 1: return run_quant_b<1, kWeight>(map, a, grid, st);
-        case 16: return run_quant_b<16, kWeight>(map, a, grid, st);
-        case 32: return run_quant_b<32, kWeight>(map, a, grid, st);
-        case 64: return run_quant_b<64, kWeight>(map, a, grid, st);
-        case 128: return run_quant_b<128, kWeight>(map, a, grid, st);
+        case 1: return run_quant_b<1, kWeight, kBf16Out>(map, a, grid, st);
+        case 16: return run_quant_b<16, kWeight, kBf16Out>(map, a, grid, st);
+        case 32: return run_quant_b<32, kWeight, kBf16Out>(map, a, grid, st);
+        case 64: return run_quant_b<64, kWeight, kBf16Out>(map, a, grid, st);
+        case 128: return run_quant_b<128, kWeight, kBf16Out>(map, a, grid, st);
         default: return MACAQ_ERR_UNSUPPORTED;
     }
 }
@@ -229,16 +230,17 @@ macaq_status run_quant_gather(int32_t b, const QuantArgs &a, const GatherArgs &g
 
 // row_index != nullptr: the gather form (activations only): output row m quantizes X row
 // row_index[m] of x_rows rows.
+// bf16_out: the transform without MXFP4 (activations only): q receives bf16 [rows, K], sf is unused.
 macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, int32_t b, bool weight,
                       const int32_t *offsets, int32_t E, uint8_t *q, uint8_t *sf, float *inv_s, cudaStream_t st,
-                      const int32_t *row_index = nullptr, int64_t x_rows = 0) {
+                      const int32_t *row_index = nullptr, int64_t x_rows = 0, bool bf16_out = false) {
     if (rows < 0 || K <= 0 || K % 128 != 0) return MACAQ_ERR_SHAPE;
     if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
     if (offsets != nullptr && (E < 1 || E > 16384)) return MACAQ_ERR_SHAPE;
     if (rows * (K / 32) >= (int64_t(1) << 31)) return MACAQ_ERR_SHAPE;
     if (row_index != nullptr && (x_rows < 1 || x_rows * K >= (int64_t(1) << 40))) return MACAQ_ERR_SHAPE;
     if (rows == 0 && (inv_s == nullptr || mul == nullptr)) return MACAQ_OK;
-    if (rows > 0 && (X == nullptr || q == nullptr || sf == nullptr)) return MACAQ_ERR_INVALID_ARG;
+    if (rows > 0 && (X == nullptr || q == nullptr || (sf == nullptr && !bf16_out))) return MACAQ_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(q) || !aligned16(sf) || !aligned16(mul) || !aligned16(inv_s) ||
         !aligned16(offsets) || !aligned16(row_index))
         return MACAQ_ERR_ALIGNMENT;
@@ -285,6 +287,7 @@ macaq_status quantize(const void *X, const float *mul, int64_t rows, int64_t K, 
         s = tensor_map(&map, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (s != MACAQ_OK) return s;
     }
+    if (bf16_out) return run_quant<false, true>(b, map, a, grid, st);
     return weight ? run_quant<true>(b, map, a, grid, st) : run_quant<false>(b, map, a, grid, st);
 }
 
@@ -710,6 +713,84 @@ macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const in
                 f.gemm_ws > 0 ? ws : nullptr, f.gemm_ws, st);
 }
 
+// ------------------------------------------------------------------------ weight-only (W4A16)
+struct WonlyLayout {
+    bool ok;
+    SkinnyPlan plan;
+    int32_t stages;
+    size_t gemm_ws, xt_off, total;
+};
+
+WonlyLayout wonly_layout(int64_t M, int64_t N, int64_t K, int sms) {
+    WonlyLayout l{};
+    if (M < 1 || M > kSkinnyMaxM || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0) return l;
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    l.plan = skinny_plan_cached(M, N, K, sms);
+    const int budget = 232448 - 1024 - 1024 - kWoTableBytes - skinny_stage_bytes_y(l.plan.mp);
+    l.stages = std::min(kWoMaxStages, budget / wo_stage_bytes(l.plan.mp));
+    l.ok = l.plan.ok && l.stages >= 2;
+    l.gemm_ws = up(l.plan.count_bytes + l.plan.partial_bytes);
+    l.xt_off = l.gemm_ws;
+    l.total = l.xt_off + up(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
+    return l;
+}
+
+macaq_status act_transform(const void *X, const float *inv_s, int64_t M, int64_t K, int32_t b, void *Xt, cudaStream_t st) {
+    return quantize(X, inv_s, M, K, b, false, nullptr, 0, static_cast<uint8_t *>(Xt), nullptr, nullptr, st, nullptr, 0,
+                    true);
+}
+
+macaq_status linear_w4a16(const void *X, const float *inv_s, int64_t M, int64_t N, int64_t K, int32_t b,
+                          const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
+                          size_t ws_bytes, cudaStream_t st) {
+    if (M < 0 || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0 || M > kSkinnyMaxM || N >= (int64_t(1) << 31))
+        return MACAQ_ERR_SHAPE;
+    if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
+    if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;
+    if (M == 0) return MACAQ_OK;
+    if (X == nullptr || Wq == nullptr || Wsf == nullptr || Y == nullptr) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(inv_s) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(Y) || !aligned16(workspace))
+        return MACAQ_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    macaq_status s = device_info(&dev);
+    if (s != MACAQ_OK) return s;
+    const WonlyLayout l = wonly_layout(M, N, K, dev.sms);
+    if (!l.ok) return MACAQ_ERR_SHAPE;
+    if (workspace == nullptr || ws_bytes < l.total) return MACAQ_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *xt = ws + l.xt_off;
+    const SkinnyPlan &p = l.plan;
+    CUtensorMap wmap, xmap, ymap;
+    s = tensor_map_2d(&wmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s == MACAQ_OK)   // X' bf16: 64-column atoms of all mp rows (rows past M read as zero)
+        s = tensor_map_2d(&xmap, xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, p.mp, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s == MACAQ_OK)
+        s = tensor_map_2d(&ymap, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, N * 2, 32, p.mp, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (s != MACAQ_OK) return s;
+    s = act_transform(X, inv_s, M, K, b, xt, st);
+    if (s != MACAQ_OK) return s;
+    SkinnyArgs g{};
+    g.y = Y;
+    g.counts = reinterpret_cast<int32_t *>(ws);
+    g.partials = reinterpret_cast<float *>(ws + p.count_bytes);
+    g.M = static_cast<int32_t>(M);
+    g.N = static_cast<int32_t>(N);
+    g.K = static_cast<int32_t>(K);
+    g.mp = p.mp;
+    g.out_f32 = out_dtype == MACAQ_OUT_F32;
+    g.stages = l.stages;
+    g.max_pieces = p.max_pieces;
+    g.units = p.units;
+    g.gran = p.gran;
+    g.wait_limit_ns = g_wait_limit_ns.load();
+    g.inv_s = nullptr;
+    const size_t smem = 1024 + static_cast<size_t>(l.stages) * wo_stage_bytes(p.mp) + kWoTableBytes +
+                        skinny_stage_bytes_y(p.mp);
+    s = set_smem(gemm_w4a16_skinny_kernel, smem);
+    if (s != MACAQ_OK) return s;
+    return launch(gemm_w4a16_skinny_kernel, dim3(p.ctas), dim3(kWoThreads), smem, st, 1, wmap, xmap, ymap, g, Wsf);
+}
+
 // ------------------------------------------------------------------------ SwiGLU -> down-projection input
 bool valid_swiglu_block(int32_t b) { return b == 1 || b == 16 || b == 32 || b == 64; }
 
@@ -948,6 +1029,26 @@ macaq_status macaq_act_quant_gather(const void *X, int64_t x_rows, const int32_t
                                        static_cast<cudaStream_t>(stream));
     return macaq::quantize(X, inv_s, M, K, had_block, false, group_offsets, E, Xq, Xsf, nullptr,
                            static_cast<cudaStream_t>(stream), row_index, x_rows);
+}
+
+macaq_status macaq_act_transform(const void *X, const float *inv_s, int64_t M, int64_t K, int32_t had_block, void *Xt,
+                                 macaq_stream_t stream) {
+    return macaq::act_transform(X, inv_s, M, K, had_block, Xt, static_cast<cudaStream_t>(stream));
+}
+
+size_t macaq_linear_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    const macaq::WonlyLayout l = macaq::wonly_layout(M, N, K, sms);
+    return l.ok ? l.total : 0;
+}
+
+macaq_status macaq_linear_w4a16(const void *X, const float *inv_s, int64_t M, int64_t N, int64_t K, int32_t had_block,
+                                const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
+                                size_t ws_bytes, macaq_stream_t stream) {
+    return macaq::linear_w4a16(X, inv_s, M, N, K, had_block, Wq, Wsf, Y, out_dtype, workspace, ws_bytes,
+                               static_cast<cudaStream_t>(stream));
 }
 
 size_t macaq_linear_swiglu_workspace_bytes(int64_t M, int64_t N, int64_t K) {

@@ -17,6 +17,8 @@
 // four neighbouring lanes combine their E8M0 bytes into one 32-bit store in the tiled SF layout.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "groups.cuh"
 #include "ptx.cuh"
 
@@ -186,6 +188,36 @@ __device__ __forceinline__ void quantize_store_group(uint64_t (&p)[16], const ui
     }
 }
 
+// The weight-only path's activation transform of one group: the per-channel multiply, the Hadamard
+// stages (activations: no 1/b), then each value rounded to bf16 (nearest even); the 64 bytes go to
+// row m, group g of a bf16 [rows, K] output (a.q reinterpreted). The whole warp calls it (shuffles).
+template <int kB>
+__device__ __forceinline__ void transform_store_bf16_group(uint64_t (&p)[16], const uint64_t (&mv)[16], const QuantArgs &a,
+                                                           bool store, uint32_t m, uint32_t g) {
+    if (a.mul != nullptr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
+    }
+    if constexpr (kB > 1) {
+        fwht_in_thread<kB>(p);
+        if constexpr (kB >= 64) fwht_cross_lane(p, 1);
+        if constexpr (kB >= 128) fwht_cross_lane(p, 2);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(a.q + (static_cast<uint64_t>(m) * a.K + g * 32) * 2);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float lo, hi;
+            upk2(p[4 * i + k], lo, hi);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+            w[k] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        if (store) dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // Zeroes the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1): groups are
 // dealt to the CTAs in turn, one warp per padding row, lanes over the 32-bit words (4 scale columns
 // each) of that row.
@@ -208,7 +240,7 @@ __device__ __forceinline__ void zero_sf_padding(const QuantArgs &a, const int32_
 // contiguous run of its row tiles, so each consumer thread owns one fixed group column and keeps that
 // column's 32 multipliers in registers (reloaded only where the expert changes). A producer warp streams the tiles with TMA (3-D tensor map rows x 128-byte chunks x
 // 64 elements, 128-byte swizzle) into a 4-stage ring with full/empty mbarriers.
-template <int kB, bool kWeight>
+template <int kB, bool kWeight, bool kBf16Out = false>
 __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a) {
     extern __shared__ uint8_t dsmem[];
     __shared__ uint64_t full_bar[kQStages];
@@ -291,11 +323,12 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[s]);
-            quantize_store_group<kB, kWeight>(p, mv, a, e, m, g, s_off, s_tb, lane);
+            if constexpr (kBf16Out) transform_store_bf16_group<kB>(p, mv, a, e >= 0, m, g);
+            else quantize_store_group<kB, kWeight>(p, mv, a, e, m, g, s_off, s_tb, lane);
         }
     }
 
-    zero_sf_padding(a, s_off, s_tb, warp, lane, kQThreads / 32);
+    if constexpr (!kBf16Out) zero_sf_padding(a, s_off, s_tb, warp, lane, kQThreads / 32);
 
     if (kWeight && a.inv_s != nullptr && a.mul != nullptr) {
         for (uint32_t k = blockIdx.x * blockDim.x + tid; k < a.K; k += gridDim.x * blockDim.x)
