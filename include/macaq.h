@@ -167,7 +167,8 @@ macaq_status macaq_act_transform(const void *X, const float *inv_s, int64_t M, i
  * with the weights prepared by macaq_prep_weights exactly as for W4A4 (codes + tiled SF) and fp32
  * accumulation on the tensor cores (kind::f16, bf16 x bf16): the weight codes are expanded to bf16
  * inside the kernel (exact for scales E8M0 <= 252) and never written to memory.
- *   X           device bf16 [M, K], 1 <= M <= 128 (M == 0 is a no-op); K % 256 == 0; N % 128 == 0
+ *   X           device bf16 [M, K], 1 <= M <= 64 (M == 0 is a no-op; larger M: MACAQ_ERR_SHAPE);
+ *               K % 256 == 0; N % 128 == 0
  *   inv_s, had_block  as for macaq_act_quant; Wq, Wsf as for macaq_linear
  *   Y           device [M, N], bf16 or fp32 per out_dtype (written)
  *   workspace   at least macaq_linear_w4a16_workspace_bytes(M, N, K) bytes (the transformed

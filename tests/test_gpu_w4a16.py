@@ -61,7 +61,7 @@ def check(X, inv, b, Wq_np, Wsf_np, repeats=1):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (3, 1024, 1024), (16, 14336 // 4, 4096), (17, 512, 2048),
-                                   (64, 1024, 5120), (128, 768, 1536)])
+                                   (64, 1024, 5120), (64, 768, 1536)])
 def test_random_codes(M, N, K):
     rng = np.random.default_rng(M + N + K)
     c = inputs.dense_case(3000 + M + N + K, M, K, 1, n_outliers=2, outlier_factor=30.0, draw_w=False)
@@ -71,6 +71,14 @@ def test_random_codes(M, N, K):
     check(c.X, inv, 32, Wq, Wsf, repeats=2)   # twice on one workspace: split counters reset themselves
 
 
+def test_larger_batches_are_refused():
+    X = torch.zeros(65, 256, dtype=torch.bfloat16, device="cuda")
+    Wq = torch.zeros(256, 128, dtype=torch.uint8, device="cuda")
+    Wsf = torch.zeros(mq.sf_bytes(256, 256), dtype=torch.uint8, device="cuda")
+    with pytest.raises(mq.MacaqError, match="MACAQ_ERR_SHAPE"):
+        mq.linear_w4a16(X, None, Wq, Wsf, had_block=1, workspace=torch.zeros(1 << 20, dtype=torch.uint8, device="cuda"))
+
+
 def test_extreme_scales_and_every_code():
     M, N, K = 4, 256, 512
     Wq = np.tile(np.arange(256, dtype=np.uint8), (N, K // 2 // 256 + 1))[:, :K // 2].copy()
@@ -78,8 +86,8 @@ def test_extreme_scales_and_every_code():
     Wsf[:, 0] = 1          # 2^-126: values down to the smallest normal bf16 / 2 (a subnormal)
     Wsf[:, 1] = 252        # 2^125: values up to 6 * 2^125, the largest the mode takes
     X = torch.zeros(M, K, dtype=torch.float32)
-    X[:, :32] = 1.0e-3     # keeps the products of the 2^125 group finite in fp32
-    X[:, 32:64] = 1.0e-30
+    X[:, :32] = 1.0e-3     # group 0 (2^-126): products below the smallest normal fp32
+    X[:, 32:64] = 1.0e-30  # group 1 (2^125): keeps its products finite in fp32
     X[:, 64:] = torch.randn(M, K - 64, generator=torch.Generator().manual_seed(3))
     check(X.to(torch.bfloat16), None, 1, Wq, Wsf)
 

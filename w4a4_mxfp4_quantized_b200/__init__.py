@@ -297,7 +297,7 @@ def act_transform(X: torch.Tensor, inv_s: torch.Tensor | None, had_block: int = 
 
 def linear_w4a16(X: torch.Tensor, inv_s: torch.Tensor | None, Wq: torch.Tensor, Wsf: torch.Tensor, *,
                  had_block: int = 32, out_dtype: int = OUT_BF16, Y=None, workspace=None):
-    """Weight-only layer for decode (M <= 128): Y = bf16(X diag(inv_s) H_b) dq(W')^T, fp32 accumulation."""
+    """Weight-only layer for decode (M <= 64): Y = bf16(X diag(inv_s) H_b) dq(W')^T, fp32 accumulation."""
     N = Wq.shape[0]
     K = Wq.shape[1] * 2
     M = X.shape[0]

@@ -723,7 +723,7 @@ struct WonlyLayout {
 
 WonlyLayout wonly_layout(int64_t M, int64_t N, int64_t K, int sms) {
     WonlyLayout l{};
-    if (M < 1 || M > kSkinnyMaxM || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0) return l;
+    if (M < 1 || M > kWoMaxM || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0) return l;
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     l.plan = skinny_plan_cached(M, N, K, sms);
     const int budget = 232448 - 1024 - 1024 - kWoTableBytes - skinny_stage_bytes_y(l.plan.mp);
@@ -743,7 +743,7 @@ macaq_status act_transform(const void *X, const float *inv_s, int64_t M, int64_t
 macaq_status linear_w4a16(const void *X, const float *inv_s, int64_t M, int64_t N, int64_t K, int32_t b,
                           const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype, void *workspace,
                           size_t ws_bytes, cudaStream_t st) {
-    if (M < 0 || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0 || M > kSkinnyMaxM || N >= (int64_t(1) << 31))
+    if (M < 0 || N <= 0 || N % 128 != 0 || K <= 0 || K % 256 != 0 || M > kWoMaxM || N >= (int64_t(1) << 31))
         return MACAQ_ERR_SHAPE;
     if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
     if (out_dtype != MACAQ_OUT_BF16 && out_dtype != MACAQ_OUT_F32) return MACAQ_ERR_INVALID_ARG;

@@ -1,4 +1,4 @@
-// w4a16.cuh -- weight-only mode: MXFP4 weights W' x bf16 activations, for decode (M <= 128).
+// w4a16.cuh -- weight-only mode: MXFP4 weights W' x bf16 activations, for decode (M <= 64).
 //
 // Page "MACaQ quantizer from huawei-csl targets GGUF, vLLM and Diffusers models" (glonce.com),
 // paragraph 3: the vLLM backend serves W4A4 or weight-only checkpoints. In the weight-only mode the
@@ -7,7 +7,7 @@
 // the MXFP4 step) but stay unquantized: rounded once to bf16, the tensor cores' operand type. So
 //     Y[m, n] = sum_k bf16(X'[m, k]) * dq(W'[n, k]),   fp32 accumulation.
 //
-// B200 mapping: the skinny swap-AB plan (W' tiles of 128 rows in the MMA's M slot, the M <= 128 rows
+// B200 mapping: the skinny swap-AB plan (W' tiles of 128 rows in the MMA's M slot, the M <= 64 rows
 // of X' in its N slot, the (tile, K-block) units split evenly over the SMs, split tiles reduced
 // through the workspace). Per 256-wide K-block the producer TMA-loads W's codes (128 rows x 128 B,
 // 128-byte swizzle), their 1 KB of scale factors and X' (four 64-column bf16 atoms, 128-byte swizzle:
@@ -24,6 +24,7 @@
 namespace macaq {
 
 constexpr int kWoMaxStages = 6;
+constexpr int kWoMaxM = 64;       // the X' atoms of more rows would leave room for fewer than 3 stages
 constexpr int kWoThreads = 320;   // producer, MMA issuer, 4 epilogue warps, 4 dequant warps
 constexpr int kWoTableBytes = 256 * 32 * 4;
 
