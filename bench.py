@@ -724,7 +724,8 @@ def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None):
     if sweep:
         out["sweep"] = " | ".join(
             f"M{p['M']}: gemm {p['gemm_us']:.1f}us {p['gemm_frac_hbm']:.2f}hbm {p['gemm_frac_fp4_peak']:.2f}fp4, "
-            f"aq {p['act_quant_us']:.1f}us, fused {p['fused_layer_us']:.1f}us" for p in sweep)
+            f"aq {p['act_quant_us']:.1f}us, fused {p['fused_layer_us']:.1f}us"
+            + (f", w4a16 {p['w4a16_layer_us']:.1f}us" if p.get("w4a16_layer_us") else "") for p in sweep)
     out["overhead"] = {k: _r(overhead[k]) for k in ("B_vs_plain_mxfp4_pipeline", "A_vs_gemm_on_prequantized_A")}
     if prefill:
         out["prefill"] = " | ".join(
@@ -812,6 +813,13 @@ def main():
         for m in M_SWEEP:
             tot, aq, gm, Lm = time_layer(m, max(10, args.steps), args.warmup, dev, dist_on, fused=True)
             fz = Lm["fused_ms"]
+            wo = None
+            if m <= 64:   # the weight-only layer on the same weights (bf16 activations)
+                ncp = len(Lm["X"])
+                Yw = torch.empty(m, N_DIM, dtype=torch.bfloat16, device=dev)
+                wo = time_graph(lambda i: mq.linear_w4a16(Lm["X"][i % ncp], Lm["inv_s"], Lm["Wq"][i % ncp],
+                                                          Lm["Wsf"][i % ncp], had_block=HAD_BLOCK, Y=Yw),
+                                max(10, args.steps), torch.cuda.current_stream(dev))
             del Lm
             fl = 2.0 * m * N_DIM * K_DIM
             g_bytes = N_DIM * K_DIM * 0.53125 + m * K_DIM * 0.53125 + m * N_DIM * 2
@@ -826,7 +834,10 @@ def main():
                           "fused_layer_us": fz * 1e3,
                           "fused_layer_tflops": fl / (fz * 1e-3) / 1e12,
                           "fused_form": "quantizer warps inside the skinny GEMM" if m <= 4
-                          else "quantizer pass + GEMM in one call"})
+                          else "quantizer pass + GEMM in one call",
+                          "w4a16_layer_us": None if wo is None else wo * 1e3,
+                          "w4a16_frac_hbm": None if wo is None else
+                          (N_DIM * K_DIM * 0.53125 + m * K_DIM * 2 + m * N_DIM * 2) / (wo * 1e-3) / 1e9 / hbm})
         prefill = prefill_section(dev, hbm, fp4_peak)
         qwen3 = qwen3_section(dev, hbm, fp4_peak)
         moe = moe_section(dev, hbm, fp4_peak)
