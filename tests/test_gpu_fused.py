@@ -137,3 +137,51 @@ def test_fused_needs_a_workspace():
                                    Wq.data_ptr(), Wsf.data_ptr(), Y.data_ptr(), mq.OUT_BF16, None, 0, st)
     assert mq.status_str(status) == "MACAQ_ERR_WORKSPACE"
     assert mq.fused_workspace_bytes(4, 256, 256) > mq.WORKSPACE_COUNTER_BYTES
+
+
+@pytest.mark.parametrize("b", [1, 16, 32, 64, 128])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 768, 1024), (2048, 14336 // 4, 4096), (4160, 1024, 8192)])
+def test_in_gemm_quantization_large_m(M, N, K, b):
+    """M > 128 with N and K multiples of 256: one launch, the 2-SM GEMM quantizes X itself (its
+    epilogue warps, between tiles) and reads A back by TMA. The result equals act_quant followed by
+    the quantized layer bit for bit, twice in a row on one workspace, and the counter region is zero
+    afterwards (4160 rows: a second, partial raster band)."""
+    c, Wq, Wsf, inv = layer(6000 + M + N + K + b, M, N, K, b, True)
+    X = c.X.cuda()
+    ref = unfused(X, inv, b, Wq, Wsf, mq.OUT_F32)
+    ref16 = unfused(X, inv, b, Wq, Wsf, mq.OUT_BF16)
+    for _ in range(2):
+        got = fused(X, inv, b, Wq, Wsf, mq.OUT_F32)
+        got16 = fused(X, inv, b, Wq, Wsf, mq.OUT_BF16)
+        torch.cuda.synchronize()
+        assert mq.device_status() == 0
+        assert torch.equal(got.view(torch.int32), ref.view(torch.int32))
+        assert torch.equal(got16.view(torch.int16), ref16.view(torch.int16))
+        assert counters_zero()
+    if b == 32:
+        rows = np.unique(np.concatenate([[0, M - 1], np.arange(127, M, 128)]))[:24]
+        check_against_oracle(c, b, True, Wq, Wsf, got, rows=rows)
+
+
+def test_in_gemm_quantization_wait_runs_out_and_resets():
+    """A 1 ns wait limit makes the producers' ready-count waits (and the pipeline waits) run out: the
+    kernel reports MACAQ_ERR_TIMEOUT, the last CTA still zeroes the counters, and the next call is
+    exact again."""
+    M, N, K = 512, 512, 1024
+    c, Wq, Wsf, inv = layer(78, M, N, K, 32, True)
+    X = c.X.cuda()
+    ref = unfused(X, inv, 32, Wq, Wsf, mq.OUT_F32)
+    torch.cuda.synchronize()
+    mq.device_status(reset=True)
+    try:
+        mq.set_wait_limit_ns(1)
+        fused(X, inv, 32, Wq, Wsf, mq.OUT_F32)
+        torch.cuda.synchronize()
+    finally:
+        mq.set_wait_limit_ns(0)
+    assert mq.device_status(reset=True) == 6
+    assert counters_zero()
+    got = fused(X, inv, 32, Wq, Wsf, mq.OUT_F32)
+    torch.cuda.synchronize()
+    assert mq.device_status() == 0
+    assert torch.equal(got.view(torch.int32), ref.view(torch.int32))

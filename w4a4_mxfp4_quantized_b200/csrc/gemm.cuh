@@ -443,6 +443,128 @@ struct PairCfg {
     static constexpr int kThreads = kGemmThreads + 32;  // + a second producer warp for the scale factors
 };
 
+// ---------------------------------------------------------------- in-kernel quantization of A
+// The fused layer (bf16 X in) for large M: the 2-SM GEMM quantizes X itself, once per element, into
+// the workspace (the same codes and scales macaq_act_quant writes) and reads A from there by TMA. The
+// work is cut into units of 16 rows x one 256-wide K-block, ordered as the GEMM's raster consumes A
+// (by band of 32 row tiles of 128, then K-block, then row tile). The epilogue warps, idle while a tile
+// accumulates, take units from a global counter whenever their own accumulator is not ready; each
+// finished unit adds one to the ready count of its (row tile, K-block), and the A and scale-factor
+// producers wait (bounded) until a K-block's count is complete before loading it. A unit never waits
+// for anything and a warp waits for its accumulator only once every unit has been handed out, so all
+// units finish. The last CTA to leave zeroes the counts and counters again (the workspace's counter
+// region is zero before and after the call). Source: aipolix.com page, paragraph 2 (the transform of
+// every layer's activations at inference).
+struct FusedA {
+    const uint16_t *x;     // bf16 [M, K]
+    const float *inv_s;    // [K] multipliers 1/s, or nullptr
+    uint8_t *xq;           // [M, K/2] codes (workspace)
+    uint8_t *xsf;          // tiled SF of M rows (workspace)
+    int32_t *flags;        // [rt_count][kb_count] finished units per (row tile, K-block)
+    int32_t *next_unit;    // units handed out
+    int32_t *exit_count;   // CTAs that have left
+    int32_t rt_count;      // ceil(M / 128)
+    int32_t kb_count;      // K / 256
+    int32_t units;         // rt_count * kb_count * kFaUnitsPerBlock
+};
+constexpr int kFaRows = 16;
+constexpr int kFaUnitsPerBlock = 128 / kFaRows;
+constexpr int kFaBandRt = 2 * kRasterM;   // 128-row tiles per raster band of the pair kernel
+
+__device__ __forceinline__ void fa_decode(const FusedA &f, int u, int &rt, int &kb, int &sub) {
+    const int full_bands = f.rt_count / kFaBandRt;
+    const int per_band = f.kb_count * kFaBandRt * kFaUnitsPerBlock;
+    int band, rem, rts;
+    if (u < full_bands * per_band) {
+        band = u / per_band;
+        rem = u - band * per_band;
+        rts = kFaBandRt;
+    } else {
+        band = full_bands;
+        rem = u - full_bands * per_band;
+        rts = f.rt_count - full_bands * kFaBandRt;
+    }
+    kb = rem / (rts * kFaUnitsPerBlock);
+    const int r2 = rem - kb * rts * kFaUnitsPerBlock;
+    rt = band * kFaBandRt + r2 / kFaUnitsPerBlock;
+    sub = r2 % kFaUnitsPerBlock;
+}
+
+// One unit by one warp: four steps of 4 rows x 8 groups (lane = row (lane / 8), group (lane % 8) of
+// the K-block, so the b >= 64 shuffles pair neighbouring groups of one row), the arithmetic of
+// macaq_act_quant; rows past M get no codes and zero scales (padding rows of the tiled SF).
+template <int kB>
+__device__ __forceinline__ void fa_quant_unit(const FusedA &f, int u, int64_t M, int K, int lane) {
+    int rt, kb, sub;
+    fa_decode(f, u, rt, kb, sub);
+    const uint32_t gcol = static_cast<uint32_t>(kb) * 8 + (lane & 7);
+    const uint32_t kq = static_cast<uint32_t>(K / 128);
+    const int64_t rows_sf = (M + 127) / 128 * 128;
+    uint64_t mv[16];
+    if (f.inv_s != nullptr) load_mul(f.inv_s + gcol * 32, mv);
+#pragma unroll 1
+    for (int step = 0; step < kFaRows / 4; ++step) {
+        const int64_t m = static_cast<int64_t>(rt) * 128 + sub * kFaRows + step * 4 + (lane >> 3);
+        uint4 raw[4];
+        if (m < M) {
+            load_group_global(f.x + m * K + gcol * 32, raw);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint64_t p[16];
+        unpack_bf16x32(raw, p);
+        if (f.inv_s != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
+        }
+        uint4 packed;
+        uint32_t E8;
+        transform_quantize_group<kB, false>(p, packed, E8);
+        if (m < M) *reinterpret_cast<uint4 *>(f.xq + m * (K / 2) + gcol * 16) = packed;
+        const uint32_t b1 = __shfl_down_sync(0xffffffffu, E8, 1);
+        const uint32_t b2 = __shfl_down_sync(0xffffffffu, E8, 2);
+        const uint32_t b3 = __shfl_down_sync(0xffffffffu, E8, 3);
+        if ((lane & 3) == 0 && m < rows_sf)
+            *reinterpret_cast<uint32_t *>(f.xsf + sf_offset(static_cast<uint32_t>(m), gcol, kq)) =
+                E8 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+    // the codes and scales are read by TMA (the async proxy) in other CTAs: order this thread's
+    // generic writes before the count that publishes them
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence();
+        atomicAdd(f.flags + rt * f.kb_count + kb, 1);
+    }
+}
+
+// Bounded wait until every unit of (row tile rt, K-block kb) has finished (row tiles past M have no
+// units); then the async proxy may read them.
+__device__ __forceinline__ bool fa_wait_ready(const FusedA &f, int rt, int kb, uint64_t limit_ns, volatile int *abort) {
+    if (rt >= f.rt_count) return true;
+    const int32_t *cnt = f.flags + rt * f.kb_count + kb;
+    auto ready = [&]() {
+        int32_t v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        return v >= kFaUnitsPerBlock;
+    };
+    if (!ready()) {
+        const uint64_t t0 = global_timer_ns();
+        while (!ready()) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                record_timeout();
+                *abort = 1;
+                return false;
+            }
+            __nanosleep(64);
+        }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
+
 // Fused SwiGLU epilogue (kSwiglu = the down projection's Hadamard block b > 0): instead of writing
 // Y, each epilogue warp takes its 32 rows x (64 gate + 64 up columns) of the accumulator, which with
 // the 64-row gate/up interleave of the weights are intermediate channels [128 nt + 64 half, + 64),
@@ -468,11 +590,12 @@ __device__ __forceinline__ void epilogue_tile_pair_swiglu(uint32_t tmem, int war
     store_swiglu64(o, static_cast<int64_t>(row0) + quarter * 32 + lane, M, c0, codes, E8);
 }
 
-template <int kSwiglu>
-__global__ void __launch_bounds__(PairCfg::kThreads, 1)
+template <int kSwiglu, int kFusedB = 0>
+__global__ void __maxnreg__(184)   // 352 threads, one CTA per SM: up to 65536 / 352 registers each
 gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                       const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
-                      const __grid_constant__ CUtensorMap ymap, GemmArgs g, int sf_replica_boxes, SwigluOut so) {
+                      const __grid_constant__ CUtensorMap ymap, GemmArgs g, int sf_replica_boxes, SwigluOut so,
+                      FusedA fa) {
     using C = PairCfg;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t dsmem[];
@@ -560,6 +683,12 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
                         stop = true;
                         break;
                     }
+                    if constexpr (kFusedB > 0) {   // A (codes or scales) of this K-block written in this launch
+                        if (!fa_wait_ready(fa, static_cast<int>(mt * 2 + rank), kb, limit, &failed)) {
+                            stop = true;
+                            break;
+                        }
+                    }
                     if (!sf) {
                         if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * C::kStageBytes);
                         tma_load_2d_pair(sA + s * C::kABytes, &amap, &full_bar[s], kb * kBKBytes, arow);
@@ -638,9 +767,26 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         uint32_t tiles_done = 0;
         uint32_t t;
         int k0, k1;
+        bool units_left = kFusedB > 0;
+        // one unit of A's quantization (fused form), unless every unit has been handed out
+        auto take_unit = [&]() {
+            if constexpr (kFusedB > 0) {
+                int u = 0;
+                if (lane == 0) u = atomicAdd(fa.next_unit, 1);
+                u = __shfl_sync(0xffffffffu, u, 0);
+                if (u >= fa.units) {
+                    units_left = false;
+                    return;
+                }
+                fa_quant_unit<kFusedB>(fa, u, g.rows, g.K, lane);
+            }
+        };
         for (uint32_t sgi = 0; segment(sgi, t, k0, k1); ++sgi, ++tiles_done) {
             uint32_t mt, nt;
             raster(t, m_tiles, n_tiles, mt, nt);
+            if constexpr (kFusedB > 0) {
+                while (units_left && !failed && !mbar_try_wait(smem_u32(&accum_full), tiles_done & 1)) take_unit();
+            }
             if (!mbar_wait_or_abort(&accum_full, tiles_done & 1, limit, &failed)) break;
             tc_fence_after();
             int leader_failed;
@@ -653,6 +799,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
                 epilogue_tile_pair(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128), static_cast<int32_t>(nt * 256),
                                    g.out_f32 != 0, &ymap, sEpi + (warp - 2) * 4096, empty_addr);
         }
+        while (units_left && !failed) take_unit();   // units other pairs still wait for
         if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it
     }
 
@@ -661,6 +808,24 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     cluster_sync();  // no CTA leaves while its partner may still touch its barriers or shared memory
     tc_fence_after();
     if (warp == 1) tmem_dealloc_pair(tmem, C::kTmemCols);
+    if constexpr (kFusedB > 0) {
+        // the last CTA to leave (every other CTA has finished its units and its waits) zeroes the
+        // ready counts and counters for the workspace's next use
+        __shared__ int s_last_cta;
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last_cta = atomicAdd(fa.exit_count, 1) == static_cast<int>(gridDim.x) - 1;
+        }
+        __syncthreads();
+        if (s_last_cta) {
+            __threadfence();
+            for (int i = threadIdx.x; i < fa.rt_count * fa.kb_count; i += blockDim.x) fa.flags[i] = 0;
+            if (threadIdx.x == 0) {
+                *fa.next_unit = 0;
+                *fa.exit_count = 0;
+            }
+        }
+    }
 }
 
 // ============================================================================ skinny (small M)

@@ -485,20 +485,22 @@ macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, i
 
 // The dense GEMM on 2-SM pairs (M > 128, N % 256 == 0, K % 256 == 0). swiglu_b > 0 selects the fused
 // SwiGLU epilogue (the down projection's quantized input goes to `so` instead of Y).
-template <int kSwiglu>
+template <int kSwiglu, int kFusedB = 0>
 macaq_status launch_pair(const CUtensorMap &amap, const CUtensorMap &bmap, const CUtensorMap &sfamap,
                          const CUtensorMap &sfbmap, const CUtensorMap &ymap, const GemmArgs &g, int replica_boxes,
-                         const SwigluOut &so, unsigned pairs, cudaStream_t st) {
-    auto k = gemm_mxf4_pair_kernel<kSwiglu>;
+                         const SwigluOut &so, const FusedA &fa, unsigned pairs, cudaStream_t st) {
+    auto k = gemm_mxf4_pair_kernel<kSwiglu, kFusedB>;
     macaq_status s = set_smem(k, PairCfg::kSmemBytes);
     if (s != MACAQ_OK) return s;
     return launch(k, dim3(2 * pairs), dim3(PairCfg::kThreads), PairCfg::kSmemBytes, st, 2, amap, bmap, sfamap, sfbmap,
-                  ymap, g, replica_boxes, so);
+                  ymap, g, replica_boxes, so, fa);
 }
 
+// fused_b > 0: A and Asf are the workspace buffers that the kernel itself fills from fa.x (the fused
+// layer's in-kernel quantization with Hadamard block fused_b).
 macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_t N, int64_t K, const uint8_t *Wq,
                       const uint8_t *Wsf, void *Y, int32_t out_dtype, const GemmArgs &g, int32_t swiglu_b,
-                      const SwigluOut &so, int sms, cudaStream_t st) {
+                      const SwigluOut &so, int sms, cudaStream_t st, int32_t fused_b = 0, const FusedA &fa = FusedA{}) {
     macaq_status s;
     CUtensorMap amap, bmap, sfamap, sfbmap;
     s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, 128,
@@ -543,12 +545,22 @@ macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_
     const int64_t tiles = ((rows + 255) / 256) * (N / 256);
     const int64_t max_pairs = sms / 2;
     const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
+    if (fused_b > 0) {
+        switch (fused_b) {
+            case 1: return launch_pair<0, 1>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+            case 16: return launch_pair<0, 16>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+            case 32: return launch_pair<0, 32>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+            case 64: return launch_pair<0, 64>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+            case 128: return launch_pair<0, 128>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+            default: return MACAQ_ERR_UNSUPPORTED;
+        }
+    }
     switch (swiglu_b) {
-        case 0: return launch_pair<0>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
-        case 1: return launch_pair<1>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
-        case 16: return launch_pair<16>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
-        case 32: return launch_pair<32>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
-        case 64: return launch_pair<64>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, pairs, st);
+        case 0: return launch_pair<0>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+        case 1: return launch_pair<1>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+        case 16: return launch_pair<16>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+        case 32: return launch_pair<32>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+        case 64: return launch_pair<64>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
         default: return MACAQ_ERR_UNSUPPORTED;
     }
 }
@@ -662,6 +674,7 @@ struct FusedLayout {
     size_t gemm_ws;   // the skinny kernel's region (counters + partials), 0 when it does not run
     size_t a_off, sf_off, total;
     bool in_kernel;   // the skinny kernel quantizes X itself
+    bool in_pair;     // the 2-SM GEMM quantizes X itself (one launch; ready counts in the counter region)
 };
 
 FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
@@ -675,6 +688,9 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
             f.in_kernel = M <= kSkinnyFusedMaxM && p.stages % 4 == 0;
         }
     }
+    // large M on 2-SM pairs: the ready counts, the work counter and the exit counter fit the region
+    f.in_pair = E == 0 && M > kSkinnyMaxM && N % 256 == 0 && K % 256 == 0 &&
+                static_cast<size_t>((M + 127) / 128) * (K / 256) + 2 <= kCountRegion / 4;
     // the activations never overlap the counter region, whichever kernel runs afterwards
     f.a_off = std::max(f.gemm_ws, up(kCountRegion));
     f.sf_off = f.a_off + up(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
@@ -707,6 +723,35 @@ macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const in
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if (offsets == nullptr && f.in_kernel)
         return run_skinny(X, nullptr, inv_s, b, M, N, K, Wq, Wsf, Y, out_dtype, ws, f.gemm_ws, dev.sms, st);
+    if (offsets == nullptr && f.in_pair) {
+        // one launch: the 2-SM GEMM quantizes X into the workspace itself (ready counts in the
+        // counter region) and reads A from there
+        FusedA fa{};
+        fa.x = static_cast<const uint16_t *>(X);
+        fa.inv_s = inv_s;
+        fa.xq = ws + f.a_off;
+        fa.xsf = ws + f.sf_off;
+        fa.rt_count = static_cast<int32_t>((M + 127) / 128);
+        fa.kb_count = static_cast<int32_t>(K / 256);
+        fa.units = fa.rt_count * fa.kb_count * kFaUnitsPerBlock;
+        int32_t *counters = reinterpret_cast<int32_t *>(ws);
+        fa.flags = counters;
+        fa.next_unit = counters + fa.rt_count * fa.kb_count;
+        fa.exit_count = fa.next_unit + 1;
+        GemmArgs g{};
+        g.asf = ws + f.sf_off;
+        g.bsf = Wsf;
+        g.y = Y;
+        g.offsets = nullptr;
+        g.rows = M;
+        g.N = static_cast<int32_t>(N);
+        g.K = static_cast<int32_t>(K);
+        g.E = 1;
+        g.out_f32 = out_dtype == MACAQ_OUT_F32;
+        g.bsf_stride = macaq_sf_bytes(N, K);
+        g.wait_limit_ns = g_wait_limit_ns.load();
+        return run_pair(ws + f.a_off, ws + f.sf_off, M, N, K, Wq, Wsf, Y, out_dtype, g, 0, SwigluOut{}, dev.sms, st, b, fa);
+    }
     s = quantize(X, inv_s, M, K, b, false, offsets, offsets != nullptr ? E : 0, ws + f.a_off, ws + f.sf_off, nullptr, st);
     if (s != MACAQ_OK) return s;
     return gemm(ws + f.a_off, ws + f.sf_off, offsets, offsets != nullptr ? E : 1, M, N, K, Wq, Wsf, Y, out_dtype,
