@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--M", type=int, default=M_MAIN)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--profile", action="store_true", help="eager passes only, for ncu captures")
+    p.add_argument("--profile-form", default="layer", choices=["layer", "fused", "w4a16"])
     p.add_argument("--details", default=None, help="also write every section's numbers to this JSON file")
     return p.parse_args()
 
@@ -606,19 +607,27 @@ def weight_prep_section(dev, hbm, steps=10):
             "gbs": b / (ms * 1e-3) / 1e9, "frac_hbm": b / (ms * 1e-3) / 1e9 / hbm}
 
 
-def profile_mode(M, steps, warmup, dev):
-    """Eager layer passes with no timing: the command the ncu captures run."""
+def profile_mode(M, steps, warmup, dev, form="layer"):
+    """Eager layer passes with no timing: the commands the ncu captures run. form: "layer" (act_quant
+    then the GEMM), "fused" (the one-call layer from bf16 X), "w4a16" (the weight-only layer)."""
     import w4a4_mxfp4_quantized_b200 as mq
 
     L = make_layer(M, dev, 2)
     for i in range(warmup + steps):
-        run_layer(mq, L, i % 2)
+        if form == "fused":
+            run_layer(mq, L, i % 2, ("fused",))
+        elif form == "w4a16":
+            mq.linear_w4a16(L["X"][i % 2], L["inv_s"], L["Wq"][i % 2], L["Wsf"][i % 2], had_block=HAD_BLOCK,
+                            Y=L["Y"][i % 2])
+        else:
+            run_layer(mq, L, i % 2)
     torch.cuda.synchronize(dev)
     assert mq.device_status() == 0
 
 
-def time_e2e(M, steps, warmup, dev, L):
-    """The same layer through the public API from pinned host X to host Y, copies included."""
+def time_e2e(M, steps, warmup, dev, L, fused=False):
+    """The same layer through the public API from pinned host X to host Y, copies included (the
+    one-call fused form when fused, else act_quant then linear)."""
     import w4a4_mxfp4_quantized_b200 as mq
 
     hX = L["host_X"].pin_memory()
@@ -628,8 +637,12 @@ def time_e2e(M, steps, warmup, dev, L):
 
     def step():
         dX.copy_(hX, non_blocking=True)
-        mq.act_quant(dX, L["inv_s"], HAD_BLOCK, Xq=L["Xq"][0], Xsf=L["Xsf"][0])
-        mq.linear(L["Xq"][0], L["Xsf"][0], L["Wq"][0], L["Wsf"][0], Y=dY)
+        if fused:
+            mq.linear(dX, None, L["Wq"][0], L["Wsf"][0], mode=mq.A_BF16_FUSED, inv_s=L["inv_s"], had_block=HAD_BLOCK,
+                      Y=dY)
+        else:
+            mq.act_quant(dX, L["inv_s"], HAD_BLOCK, Xq=L["Xq"][0], Xsf=L["Xsf"][0])
+            mq.linear(L["Xq"][0], L["Xsf"][0], L["Wq"][0], L["Wsf"][0], Y=dY)
         hY.copy_(dY, non_blocking=True)
 
     for _ in range(warmup):
@@ -726,7 +739,8 @@ def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None):
             f"M{p['M']}: gemm {p['gemm_us']:.1f}us {p['gemm_frac_hbm']:.2f}hbm {p['gemm_frac_fp4_peak']:.2f}fp4, "
             f"aq {p['act_quant_us']:.1f}us, fused {p['fused_layer_us']:.1f}us"
             + (f", w4a16 {p['w4a16_layer_us']:.1f}us" if p.get("w4a16_layer_us") else "") for p in sweep)
-    out["overhead"] = {k: _r(overhead[k]) for k in ("B_vs_plain_mxfp4_pipeline", "A_vs_gemm_on_prequantized_A")}
+    out["overhead"] = {k: _r(overhead[k]) for k in ("B_vs_plain_mxfp4_pipeline", "A_vs_gemm_on_prequantized_A",
+                                                     "two_kernel_B")}
     if prefill:
         out["prefill"] = " | ".join(
             f"{p['M']}x{p['K']}x{p['N']}: gemm {p['gemm_ms']:.3f}ms {p['gemm_frac_fp4_peak']:.2f}fp4, "
@@ -784,29 +798,39 @@ def main():
 
     M = args.M
     if args.profile:
-        profile_mode(M, args.steps, args.warmup, dev)
+        profile_mode(M, args.steps, args.warmup, dev, args.profile_form)
         return
     flops = 2.0 * M * N_DIM * K_DIM
     with ClockSampler(local) as clk:
-        total_ms, aq_ms, gemm_ms, L = time_layer(M, args.steps, args.warmup, dev, dist_on)
+        total_ms, aq_ms, gemm_ms, L = time_layer(M, args.steps, args.warmup, dev, dist_on, fused=True)
     clocks = clk.summary()
-    ms_step = max_over_ranks(total_ms, dist_on, dev) / args.steps
+    two_kernel_ms = total_ms / args.steps
+    fused_ms = L["fused_ms"]
+    # the step is the faster of the library's two forms of the layer: act_quant then the GEMM (two
+    # launches), or the one call from bf16 X (one launch for large M: the GEMM quantizes X itself)
+    fused_step = fused_ms < two_kernel_ms
+    ms_step = max_over_ranks(fused_ms if fused_step else two_kernel_ms, dist_on, dev)
     value = job_tflops(world, flops, ms_step)
 
     del L
-    p_total, p_aq, p_gemm, _ = time_layer(M, args.steps, args.warmup, dev, dist_on, plain=True)
-    overhead = {"plain_mxfp4_ms_per_step": p_total / args.steps, "plain_act_quant_ms": p_aq, "plain_gemm_ms": p_gemm,
-                "B_vs_plain_mxfp4_pipeline": (total_ms / args.steps) / (p_total / args.steps) - 1.0,
-                "A_vs_gemm_on_prequantized_A": (total_ms / args.steps) / p_gemm - 1.0,
+    p_total, p_aq, p_gemm, Lp = time_layer(M, args.steps, args.warmup, dev, dist_on, plain=True, fused=True)
+    p_fused = Lp["fused_ms"]
+    del Lp
+    p_step = p_fused if fused_step else p_total / args.steps
+    overhead = {"plain_mxfp4_ms_per_step": p_step, "plain_act_quant_ms": p_aq, "plain_gemm_ms": p_gemm,
+                "B_vs_plain_mxfp4_pipeline": ms_step / p_step - 1.0,
+                "A_vs_gemm_on_prequantized_A": ms_step / p_gemm - 1.0,
+                "two_kernel_B": two_kernel_ms / (p_total / args.steps) - 1.0,
                 "pages_figure_for_context": "2.3% end-to-end, Qwen3-32B in vLLM, hardware not stated"}
     _, _, _, L = time_layer(M, 3, 1, dev, dist_on)
-    e2e_ms, h2d, d2h = time_e2e(M, max(3, args.steps // 2), 2, dev, L)
+    e2e_ms, h2d, d2h = time_e2e(M, max(3, args.steps // 2), 2, dev, L, fused_step)
     del L
     e2e_ms = max_over_ranks(e2e_ms, dist_on, dev)
     e2e_value = job_tflops(world, flops, e2e_ms)
 
-    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
-    gemm_kernel = gemm_kernel_name(M)
+    # the dominant kernel: the GEMM, or in the one-launch form the GEMM that also quantizes X
+    gemm_tflops = flops / ((fused_ms if fused_step else gemm_ms) * 1e-3) / 1e12
+    gemm_kernel = gemm_kernel_name(M) + (" (one launch, quantizing X itself)" if fused_step else "")
     aq_bytes = M * K_DIM * (2 + 0.5 + 1 / 32)
     sweep, prefill, qwen3, moe, prep, ceiling, flip = [], None, None, None, None, [], None
     if not args.no_sweep:
@@ -834,7 +858,7 @@ def main():
                           "fused_layer_us": fz * 1e3,
                           "fused_layer_tflops": fl / (fz * 1e-3) / 1e12,
                           "fused_form": "quantizer warps inside the skinny GEMM" if m <= 4
-                          else "quantizer pass + GEMM in one call",
+                          else ("quantizer pass + skinny GEMM" if m <= 128 else "2-SM GEMM quantizing X itself (one launch)"),
                           "w4a16_layer_us": None if wo is None else wo * 1e3,
                           "w4a16_frac_hbm": None if wo is None else
                           (N_DIM * K_DIM * 0.53125 + m * K_DIM * 2 + m * N_DIM * 2) / (wo * 1e-3) / 1e9 / hbm})
@@ -861,14 +885,16 @@ def main():
         "act_quant_roofline": {"kernel": "quant_kernel", "bound": "hbm", "achieved": aq_bytes / (aq_ms * 1e-3) / 1e9,
                                "peak": hbm, "unit": "GB/s", "frac": aq_bytes / (aq_ms * 1e-3) / 1e9 / hbm,
                                "peak_source": peak_src, "traffic": profiled_traffic("quant_kernel", M)},
-        "kernel_ms": {"act_quant": aq_ms, "gemm": gemm_ms},
-        "gpu_launches": 2 * args.steps,
+        "kernel_ms": {"act_quant": aq_ms, "gemm": gemm_ms, "two_kernel_step": two_kernel_ms, "one_call_step": fused_ms},
+        "form": "one call (bf16 X in, in-GEMM quantization)" if fused_step else "act_quant + GEMM",
+        "gpu_launches": (1 if fused_step else 2) * args.steps,
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "clocks": dict(clocks, window="warm replays (1.5 s of this workload) and the timed replay"),
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
     out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip)
+    out["summary"]["gemm_alone"] = f"{gemm_ms * 1e3:.1f}us {flops / (gemm_ms * 1e-3) / 1e12 / fp4_peak:.3f}fp4 (pre-quantized A)"
     if args.details:
         with open(args.details, "w") as f:
             json.dump({**out, "sweep": sweep, "transform_overhead": overhead, "prefill": prefill, "qwen3": qwen3,

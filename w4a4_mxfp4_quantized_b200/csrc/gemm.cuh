@@ -591,7 +591,7 @@ __device__ __forceinline__ void epilogue_tile_pair_swiglu(uint32_t tmem, int war
 }
 
 template <int kSwiglu, int kFusedB = 0>
-__global__ void __maxnreg__(184)   // 352 threads, one CTA per SM: up to 65536 / 352 registers each
+__global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                       const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
                       const __grid_constant__ CUtensorMap ymap, GemmArgs g, int sf_replica_boxes, SwigluOut so,
