@@ -74,7 +74,7 @@ typedef enum { MACAQ_OUT_BF16 = 0, MACAQ_OUT_F32 = 1 } macaq_out_dtype;
 
 /* How operand A of the GEMM is given: already quantized (codes + SF from macaq_act_quant), or as
  * bf16 activations that the GEMM transforms and quantizes itself (the fused variant). */
-typedef enum { MACAQ_A_QUANTIZED = 0, MACAQ_A_BF16_FUSED = 1 } macaq_a_mode;
+typedef enum { MACAQ_A_QUANTIZED = 0, MACAQ_A_BF16_FUSED = 1, MACAQ_A_BF16_ONE_LAUNCH = 2 } macaq_a_mode;
 
 /* A cudaStream_t, passed as a plain pointer so that this header needs no CUDA include. */
 typedef void *macaq_stream_t;
@@ -251,6 +251,14 @@ macaq_status macaq_moe_combine(const void *Y, int64_t y_rows, int64_t N, const i
  *                               quantized activation in HBM). Otherwise: a quantizer pass into the
  *                               workspace, then the GEMM, in stream order. Needs a workspace of
  *                               macaq_fused_workspace_bytes(M, N, K, 0) bytes (else MACAQ_ERR_WORKSPACE).
+ *   mode == MACAQ_A_BF16_ONE_LAUNCH: as MACAQ_A_BF16_FUSED (same arguments, workspace and result),
+ *                               but M > 128 with N % 256 == 0 and K % 256 == 0 runs as ONE launch: the
+ *                               2-SM GEMM's epilogue warps quantize X into the workspace between tiles
+ *                               and its producers wait (bounded) on per-block ready counts before
+ *                               loading A. On B200 this form measures slower than the two launches
+ *                               (the epilogue warps quantize at about half the quantizer kernel's
+ *                               rate, and the first tiles wait for them), which is why it is not the
+ *                               default; other shapes behave exactly as MACAQ_A_BF16_FUSED.
  *   Wq, Wsf    from macaq_prep_weights: u8 [N, K/2] and the tiled SF of N rows
  *   Y          device [M, N], bf16 or fp32 per out_dtype (written)
  *   workspace  NULL, or device scratch of at least macaq_workspace_bytes(M, N, K, 0) bytes under the

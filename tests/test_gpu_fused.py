@@ -4,6 +4,8 @@ The quantization is bit-exact and the GEMM plan is the same as for the quantized
 result must equal act_quant followed by the quantized linear bit for bit; it is also checked against
 the oracle's pipeline (oracle act_quant, float64 GEMM) within 1e-5 of sum|terms| per element. M <= 4
 with K % 256 == 0 runs the quantizer inside the skinny GEMM kernel; larger M runs the two-pass form.
+Mode A_BF16_ONE_LAUNCH gives the same result; for M > 128 the 2-SM GEMM quantizes X itself in one
+launch.
 """
 import ctypes
 
@@ -31,8 +33,8 @@ def unfused(X, inv, b, Wq, Wsf, out_dtype):
     return mq.linear(Xq, Xsf, Wq, Wsf, out_dtype=out_dtype)
 
 
-def fused(X, inv, b, Wq, Wsf, out_dtype):
-    return mq.linear(X, None, Wq, Wsf, mode=mq.A_BF16_FUSED, inv_s=inv, had_block=b, out_dtype=out_dtype)
+def fused(X, inv, b, Wq, Wsf, out_dtype, mode=mq.A_BF16_FUSED):
+    return mq.linear(X, None, Wq, Wsf, mode=mode, inv_s=inv, had_block=b, out_dtype=out_dtype)
 
 
 def counters_zero():
@@ -140,19 +142,22 @@ def test_fused_needs_a_workspace():
 
 
 @pytest.mark.parametrize("b", [1, 16, 32, 64, 128])
-@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 768, 1024), (2048, 14336 // 4, 4096), (4160, 1024, 8192)])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 768, 1024), (2048, 14336 // 4, 4096), (4160, 1024, 8192),
+                                   (2048, 14336, 512), (1300, 14336, 1024)])
 def test_in_gemm_quantization_large_m(M, N, K, b):
-    """M > 128 with N and K multiples of 256: one launch, the 2-SM GEMM quantizes X itself (its
+    """Mode A_BF16_ONE_LAUNCH, M > 128 with N and K multiples of 256: one launch, the 2-SM GEMM quantizes X itself (its
     epilogue warps, between tiles) and reads A back by TMA. The result equals act_quant followed by
     the quantized layer bit for bit, twice in a row on one workspace, and the counter region is zero
-    afterwards (4160 rows: a second, partial raster band)."""
+    afterwards. N = 14336 gives 56 column tiles, so the host cuts the raster into bands of three
+    256-row tiles: 2048 rows make three bands (the last one of two), 1300 rows two bands with a
+    partial last row tile; 4160 rows at N = 1024 make a second, partial band of the default height."""
     c, Wq, Wsf, inv = layer(6000 + M + N + K + b, M, N, K, b, True)
     X = c.X.cuda()
     ref = unfused(X, inv, b, Wq, Wsf, mq.OUT_F32)
     ref16 = unfused(X, inv, b, Wq, Wsf, mq.OUT_BF16)
     for _ in range(2):
-        got = fused(X, inv, b, Wq, Wsf, mq.OUT_F32)
-        got16 = fused(X, inv, b, Wq, Wsf, mq.OUT_BF16)
+        got = fused(X, inv, b, Wq, Wsf, mq.OUT_F32, mq.A_BF16_ONE_LAUNCH)
+        got16 = fused(X, inv, b, Wq, Wsf, mq.OUT_BF16, mq.A_BF16_ONE_LAUNCH)
         torch.cuda.synchronize()
         assert mq.device_status() == 0
         assert torch.equal(got.view(torch.int32), ref.view(torch.int32))
@@ -175,13 +180,13 @@ def test_in_gemm_quantization_wait_runs_out_and_resets():
     mq.device_status(reset=True)
     try:
         mq.set_wait_limit_ns(1)
-        fused(X, inv, 32, Wq, Wsf, mq.OUT_F32)
+        fused(X, inv, 32, Wq, Wsf, mq.OUT_F32, mq.A_BF16_ONE_LAUNCH)
         torch.cuda.synchronize()
     finally:
         mq.set_wait_limit_ns(0)
     assert mq.device_status(reset=True) == 6
     assert counters_zero()
-    got = fused(X, inv, 32, Wq, Wsf, mq.OUT_F32)
+    got = fused(X, inv, 32, Wq, Wsf, mq.OUT_F32, mq.A_BF16_ONE_LAUNCH)
     torch.cuda.synchronize()
     assert mq.device_status() == 0
     assert torch.equal(got.view(torch.int32), ref.view(torch.int32))

@@ -21,7 +21,7 @@ import threading
 import torch
 
 __all__ = [
-    "MacaqError", "OUT_BF16", "OUT_F32", "A_QUANTIZED", "A_BF16_FUSED",
+    "MacaqError", "OUT_BF16", "OUT_F32", "A_QUANTIZED", "A_BF16_FUSED", "A_BF16_ONE_LAUNCH",
     "sf_bytes", "grouped_sf_bytes", "workspace_bytes", "fused_workspace_bytes", "WORKSPACE_COUNTER_BYTES",
     "status_str",
     "prep_weights", "act_quant", "linear", "linear_fixed_scratch", "grouped_linear", "device_status",
@@ -37,7 +37,7 @@ _lib = None
 
 OUT_BF16, OUT_F32 = 0, 1
 WORKSPACE_COUNTER_BYTES = 65536  # MACAQ_WORKSPACE_COUNTER_BYTES: the zero-between-calls counter region
-A_QUANTIZED, A_BF16_FUSED = 0, 1
+A_QUANTIZED, A_BF16_FUSED, A_BF16_ONE_LAUNCH = 0, 1, 2
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -328,13 +328,15 @@ def linear(A: torch.Tensor, Asf: torch.Tensor | None, Wq: torch.Tensor, Wsf: tor
     kernel (weights in the MMA's M slot, split over all SMs); use_workspace=False runs the general
     kernel instead.
     mode=A_BF16_FUSED: A is bf16 X [M, K]; the call applies inv_s, H_b and MXFP4 itself (inside the
-    GEMM kernel for M <= 4) and needs a workspace."""
+    GEMM kernel for M <= 4, else a quantizer pass then the GEMM) and needs a workspace.
+    mode=A_BF16_ONE_LAUNCH: the same result; M > 128 (N, K % 256 == 0) runs as one launch in which
+    the 2-SM GEMM quantizes X itself."""
     N = Wq.shape[0]
     K = Wq.shape[1] * 2
     M = A.shape[0]
     dev = A.device
     Y = _out(M, N, out_dtype, dev, Y)
-    fused = mode == A_BF16_FUSED
+    fused = mode in (A_BF16_FUSED, A_BF16_ONE_LAUNCH)
     if fused:
         ws_need = fused_workspace_bytes(M, N, K, 0)
     else:

@@ -70,6 +70,7 @@ struct GemmArgs {
     int32_t out_f32;
     uint64_t bsf_stride;       // bytes between experts' SF
     uint64_t wait_limit_ns;
+    int32_t raster_m;          // 2-SM kernel: 256-row tiles per raster band (<= 0: kRasterM)
 };
 
 template <int BN>
@@ -94,14 +95,18 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parit
     }
 }
 
-// Tile index -> (row tile, column tile) in bands of kRasterM row tiles, columns inner.
-__device__ __forceinline__ void raster(uint32_t t, uint32_t m_tiles, uint32_t n_tiles, uint32_t &mt, uint32_t &nt) {
-    const uint32_t band = t / (kRasterM * n_tiles);
-    const uint32_t first = band * kRasterM;
-    const uint32_t height = min(static_cast<uint32_t>(kRasterM), m_tiles - first);
-    const uint32_t r = t - band * kRasterM * n_tiles;
+// Tile index -> (row tile, column tile) in bands of `bm` row tiles, columns inner.
+__device__ __forceinline__ void raster(uint32_t t, uint32_t m_tiles, uint32_t n_tiles, uint32_t bm, uint32_t &mt,
+                                       uint32_t &nt) {
+    const uint32_t band = t / (bm * n_tiles);
+    const uint32_t first = band * bm;
+    const uint32_t height = min(bm, m_tiles - first);
+    const uint32_t r = t - band * bm * n_tiles;
     mt = first + r % height;
     nt = r / height;
+}
+__device__ __forceinline__ void raster(uint32_t t, uint32_t m_tiles, uint32_t n_tiles, uint32_t &mt, uint32_t &nt) {
+    raster(t, m_tiles, n_tiles, kRasterM, mt, nt);
 }
 
 // Epilogue of one output tile for one epilogue warp. Warp w (2..9) reads TMEM lane quarter w % 4
@@ -447,10 +452,15 @@ struct PairCfg {
 // The fused layer (bf16 X in) for large M: the 2-SM GEMM quantizes X itself, once per element, into
 // the workspace (the same codes and scales macaq_act_quant writes) and reads A from there by TMA. The
 // work is cut into units of 16 rows x one 256-wide K-block, ordered as the GEMM's raster consumes A
-// (by band of 32 row tiles of 128, then K-block, then row tile). The epilogue warps, idle while a tile
-// accumulates, take units from a global counter whenever their own accumulator is not ready; each
-// finished unit adds one to the ready count of its (row tile, K-block), and the A and scale-factor
-// producers wait (bounded) until a K-block's count is complete before loading it. A unit never waits
+// (by raster band, then K-block, then row tile). The host picks a low band (about two rounds of
+// tiles per band) so that the first tiles need only the first band's rows: its units are taken by
+// the idle epilogue warps at once, and later bands are quantized while earlier tiles accumulate. The epilogue warps, idle while a tile
+// accumulates, take units whenever their own accumulator is not ready (the first one by warp index,
+// the rest from a global counter); each
+// finished unit adds one to the ready count of its (row tile, K-block) and to that of its row tile.
+// At the start of a tile the A and scale-factor producers read the row tile's count once: when it is
+// complete they load every K-block without further checks, otherwise they wait (bounded) for each
+// K-block's count to complete before loading it, reading the counts of several K-blocks per trip. A unit never waits
 // for anything and a warp waits for its accumulator only once every unit has been handed out, so all
 // units finish. The last CTA to leave zeroes the counts and counters again (the workspace's counter
 // region is zero before and after the call). Source: aipolix.com page, paragraph 2 (the transform of
@@ -461,38 +471,40 @@ struct FusedA {
     uint8_t *xq;           // [M, K/2] codes (workspace)
     uint8_t *xsf;          // tiled SF of M rows (workspace)
     int32_t *flags;        // [rt_count][kb_count] finished units per (row tile, K-block)
+    int32_t *rt_done;      // [rt_count] finished units per row tile (all K-blocks)
     int32_t *next_unit;    // units handed out
     int32_t *exit_count;   // CTAs that have left
     int32_t rt_count;      // ceil(M / 128)
     int32_t kb_count;      // K / 256
     int32_t units;         // rt_count * kb_count * kFaUnitsPerBlock
+    int32_t band_rt;       // 128-row tiles per raster band of the GEMM (2 x its band of 256-row tiles)
 };
 constexpr int kFaRows = 16;
 constexpr int kFaUnitsPerBlock = 128 / kFaRows;
-constexpr int kFaBandRt = 2 * kRasterM;   // 128-row tiles per raster band of the pair kernel
 
 __device__ __forceinline__ void fa_decode(const FusedA &f, int u, int &rt, int &kb, int &sub) {
-    const int full_bands = f.rt_count / kFaBandRt;
-    const int per_band = f.kb_count * kFaBandRt * kFaUnitsPerBlock;
+    const int full_bands = f.rt_count / f.band_rt;
+    const int per_band = f.kb_count * f.band_rt * kFaUnitsPerBlock;
     int band, rem, rts;
     if (u < full_bands * per_band) {
         band = u / per_band;
         rem = u - band * per_band;
-        rts = kFaBandRt;
+        rts = f.band_rt;
     } else {
         band = full_bands;
         rem = u - full_bands * per_band;
-        rts = f.rt_count - full_bands * kFaBandRt;
+        rts = f.rt_count - full_bands * f.band_rt;
     }
     kb = rem / (rts * kFaUnitsPerBlock);
     const int r2 = rem - kb * rts * kFaUnitsPerBlock;
-    rt = band * kFaBandRt + r2 / kFaUnitsPerBlock;
+    rt = band * f.band_rt + r2 / kFaUnitsPerBlock;
     sub = r2 % kFaUnitsPerBlock;
 }
 
-// One unit by one warp: four steps of 4 rows x 8 groups (lane = row (lane / 8), group (lane % 8) of
-// the K-block, so the b >= 64 shuffles pair neighbouring groups of one row), the arithmetic of
-// macaq_act_quant; rows past M get no codes and zero scales (padding rows of the tiled SF).
+// One unit by one warp: kFaRows / 4 steps of 4 rows x 8 groups (lane = row (lane / 8), group
+// (lane % 8) of the K-block, so the b >= 64 shuffles pair neighbouring groups of one row), the
+// arithmetic of macaq_act_quant; rows past M get no codes and zero scales (padding rows of the tiled
+// SF). All steps' loads are issued before the first step's arithmetic: one trip to memory per unit.
 template <int kB>
 __device__ __forceinline__ void fa_quant_unit(const FusedA &f, int u, int64_t M, int K, int lane) {
     int rt, kb, sub;
@@ -500,20 +512,25 @@ __device__ __forceinline__ void fa_quant_unit(const FusedA &f, int u, int64_t M,
     const uint32_t gcol = static_cast<uint32_t>(kb) * 8 + (lane & 7);
     const uint32_t kq = static_cast<uint32_t>(K / 128);
     const int64_t rows_sf = (M + 127) / 128 * 128;
-    uint64_t mv[16];
-    if (f.inv_s != nullptr) load_mul(f.inv_s + gcol * 32, mv);
-#pragma unroll 1
+    const int64_t m0 = static_cast<int64_t>(rt) * 128 + sub * kFaRows + (lane >> 3);
+    uint4 raw[kFaRows / 4][4];
+#pragma unroll
     for (int step = 0; step < kFaRows / 4; ++step) {
-        const int64_t m = static_cast<int64_t>(rt) * 128 + sub * kFaRows + step * 4 + (lane >> 3);
-        uint4 raw[4];
+        const int64_t m = m0 + step * 4;
         if (m < M) {
-            load_group_global(f.x + m * K + gcol * 32, raw);
+            load_group_global(f.x + m * K + gcol * 32, raw[step]);
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < 4; ++i) raw[step][i] = make_uint4(0u, 0u, 0u, 0u);
         }
+    }
+    uint64_t mv[16];
+    if (f.inv_s != nullptr) load_mul(f.inv_s + gcol * 32, mv);
+#pragma unroll
+    for (int step = 0; step < kFaRows / 4; ++step) {
+        const int64_t m = m0 + step * 4;
         uint64_t p[16];
-        unpack_bf16x32(raw, p);
+        unpack_bf16x32(raw[step], p);
         if (f.inv_s != nullptr) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
@@ -530,39 +547,65 @@ __device__ __forceinline__ void fa_quant_unit(const FusedA &f, int u, int64_t M,
                 E8 | (b1 << 8) | (b2 << 16) | (b3 << 24);
     }
     // the codes and scales are read by TMA (the async proxy) in other CTAs: order this thread's
-    // generic writes before the count that publishes them
+    // generic writes before the counts that publish them
     asm volatile("fence.proxy.async.global;" ::: "memory");
     __syncwarp();
     if (lane == 0) {
         __threadfence();
         atomicAdd(f.flags + rt * f.kb_count + kb, 1);
+        atomicAdd(f.rt_done + rt, 1);
     }
 }
 
-// Bounded wait until every unit of (row tile rt, K-block kb) has finished (row tiles past M have no
-// units); then the async proxy may read them.
-__device__ __forceinline__ bool fa_wait_ready(const FusedA &f, int rt, int kb, uint64_t limit_ns, volatile int *abort) {
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// True when every unit of row tile rt (all K-blocks) has finished; row tiles past M have no units.
+// Then the async proxy may read all of the row tile's codes and scales.
+__device__ __forceinline__ bool fa_row_tile_ready(const FusedA &f, int rt) {
     if (rt >= f.rt_count) return true;
-    const int32_t *cnt = f.flags + rt * f.kb_count + kb;
-    auto ready = [&]() {
-        int32_t v;
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        return v >= kFaUnitsPerBlock;
-    };
-    if (!ready()) {
-        const uint64_t t0 = global_timer_ns();
-        while (!ready()) {
-            if (*abort) return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                record_timeout();
-                *abort = 1;
-                return false;
-            }
-            __nanosleep(64);
-        }
-    }
+    if (ld_acquire_gpu(f.rt_done + rt) < f.kb_count * kFaUnitsPerBlock) return false;
     asm volatile("fence.proxy.async.global;" ::: "memory");
     return true;
+}
+
+// Bounded wait until K-block kb of row tile rt has all its units finished (row tiles past M have
+// none). The counts of up to kFaPeek K-blocks from kb are read together (relaxed loads, then one
+// acquire fence), so a run of finished K-blocks costs one trip to L2; returns the end of the run of
+// finished K-blocks (> kb), or -1 when the wait ran out or another role failed. Then the async proxy
+// may read those K-blocks.
+constexpr int kFaPeek = 8;
+__device__ __forceinline__ int fa_wait_ready(const FusedA &f, int rt, int kb, uint64_t limit_ns, volatile int *abort) {
+    if (rt >= f.rt_count) return f.kb_count;
+    const int32_t *cnt = f.flags + rt * f.kb_count;
+    const int n = min(kFaPeek, f.kb_count - kb);
+    uint64_t t0 = 0;
+    while (true) {
+        int32_t v[kFaPeek];
+#pragma unroll
+        for (int i = 0; i < kFaPeek; ++i)
+            if (i < n) asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v[i]) : "l"(cnt + kb + i) : "memory");
+        int run = 0;
+#pragma unroll
+        for (int i = 0; i < kFaPeek; ++i)
+            if (i < n && run == i && v[i] >= kFaUnitsPerBlock) run = i + 1;
+        if (run > 0) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return kb + run;
+        }
+        if (*abort) return -1;
+        if (t0 == 0) t0 = global_timer_ns();
+        else if (global_timer_ns() - t0 > limit_ns) {
+            record_timeout();
+            *abort = 1;
+            return -1;
+        }
+        __nanosleep(64);
+    }
 }
 
 // Fused SwiGLU epilogue (kSwiglu = the down projection's Hadamard block b > 0): instead of writing
@@ -621,6 +664,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     const uint32_t m_tiles = static_cast<uint32_t>((g.rows + 255) / 256);
     const uint32_t n_tiles = static_cast<uint32_t>(g.N / 256);
     const uint32_t num_tiles = m_tiles * n_tiles;  // the host launches at most this many pairs
+    const uint32_t band_m = g.raster_m > 0 ? static_cast<uint32_t>(g.raster_m) : static_cast<uint32_t>(kRasterM);
     const int K = g.K;
     const int kq = K / 128;
     const int num_kb = K / 256;
@@ -672,11 +716,16 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
             int k0, k1;
             for (uint32_t sgi = 0; !stop && segment(sgi, t, k0, k1); ++sgi) {
                 uint32_t mt, nt;
-                raster(t, m_tiles, n_tiles, mt, nt);
+                raster(t, m_tiles, n_tiles, band_m, mt, nt);
                 const int32_t arow = static_cast<int32_t>(mt * 256 + rank * 128);
                 const int32_t brow = static_cast<int32_t>(nt * 256 + rank * 128);
                 const int32_t a_tile = static_cast<int32_t>((mt * 2 + rank) * kq);   // first 128x4 tile of A's rows
                 const int32_t b_tile = static_cast<int32_t>(nt * 2 * kq);            // of B's first 128 rows
+                // fused form: once the row tile's units have all finished, its K-blocks need no checks;
+                // otherwise a_ready_end is the end of the run of K-blocks known to be finished
+                int a_ready_end = num_kb;
+                if constexpr (kFusedB > 0)
+                    if (!fa_row_tile_ready(fa, static_cast<int>(mt * 2 + rank))) a_ready_end = 0;
                 for (int kb = k0; kb < k1; ++kb, ++j) {
                     const int s = j % S;
                     if (j >= S && !mbar_wait_or_abort(&empty_bar[s], ((j / S) & 1) ^ 1, limit, &failed)) {
@@ -684,9 +733,12 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
                         break;
                     }
                     if constexpr (kFusedB > 0) {   // A (codes or scales) of this K-block written in this launch
-                        if (!fa_wait_ready(fa, static_cast<int>(mt * 2 + rank), kb, limit, &failed)) {
-                            stop = true;
-                            break;
+                        if (kb >= a_ready_end) {
+                            a_ready_end = fa_wait_ready(fa, static_cast<int>(mt * 2 + rank), kb, limit, &failed);
+                            if (a_ready_end < 0) {
+                                stop = true;
+                                break;
+                            }
                         }
                     }
                     if (!sf) {
@@ -768,12 +820,19 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         uint32_t t;
         int k0, k1;
         bool units_left = kFusedB > 0;
-        // one unit of A's quantization (fused form), unless every unit has been handed out
+        // one unit of A's quantization (fused form), unless every unit has been handed out. Epilogue
+        // warp w of the launch takes unit w first (all of them start idle, so no counter is needed);
+        // later units come from the shared counter, past the first gridDim.x * kEpiWarps
+        const int first_unit = static_cast<int>(blockIdx.x) * kEpiWarps + (warp - 2);
+        bool took_first = false;
         auto take_unit = [&]() {
             if constexpr (kFusedB > 0) {
-                int u = 0;
-                if (lane == 0) u = atomicAdd(fa.next_unit, 1);
-                u = __shfl_sync(0xffffffffu, u, 0);
+                int u = first_unit;
+                if (took_first) {
+                    if (lane == 0) u = static_cast<int>(gridDim.x) * kEpiWarps + atomicAdd(fa.next_unit, 1);
+                    u = __shfl_sync(0xffffffffu, u, 0);
+                }
+                took_first = true;
                 if (u >= fa.units) {
                     units_left = false;
                     return;
@@ -783,9 +842,11 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         };
         for (uint32_t sgi = 0; segment(sgi, t, k0, k1); ++sgi, ++tiles_done) {
             uint32_t mt, nt;
-            raster(t, m_tiles, n_tiles, mt, nt);
+            raster(t, m_tiles, n_tiles, band_m, mt, nt);
             if constexpr (kFusedB > 0) {
-                while (units_left && !failed && !mbar_try_wait(smem_u32(&accum_full), tiles_done & 1)) take_unit();
+                // test_wait, not try_wait: a blocking poll would hold the warp for the suspend limit
+                // between units while the accumulator is far from ready
+                while (units_left && !failed && !mbar_test_wait(smem_u32(&accum_full), tiles_done & 1)) take_unit();
             }
             if (!mbar_wait_or_abort(&accum_full, tiles_done & 1, limit, &failed)) break;
             tc_fence_after();
@@ -820,6 +881,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         if (s_last_cta) {
             __threadfence();
             for (int i = threadIdx.x; i < fa.rt_count * fa.kb_count; i += blockDim.x) fa.flags[i] = 0;
+            for (int i = threadIdx.x; i < fa.rt_count; i += blockDim.x) fa.rt_done[i] = 0;
             if (threadIdx.x == 0) {
                 *fa.next_unit = 0;
                 *fa.exit_count = 0;

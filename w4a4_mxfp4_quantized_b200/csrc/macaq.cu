@@ -546,12 +546,20 @@ macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_
     const int64_t max_pairs = sms / 2;
     const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
     if (fused_b > 0) {
+        // in-GEMM quantization: raster bands of about two rounds of tiles, so the first round needs
+        // only the first band's rows of A; the units follow the same bands
+        const int64_t n_tiles = N / 256;
+        const int64_t band = std::min<int64_t>(kRasterM, std::max<int64_t>(2, (2 * pairs + n_tiles - 1) / n_tiles));
+        GemmArgs gb = g;
+        gb.raster_m = static_cast<int32_t>(band);
+        FusedA fb = fa;
+        fb.band_rt = static_cast<int32_t>(2 * band);
         switch (fused_b) {
-            case 1: return launch_pair<0, 1>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
-            case 16: return launch_pair<0, 16>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
-            case 32: return launch_pair<0, 32>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
-            case 64: return launch_pair<0, 64>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
-            case 128: return launch_pair<0, 128>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
+            case 1: return launch_pair<0, 1>(amap, bmap, sfamap, sfbmap, ymap, gb, replica_boxes, so, fb, pairs, st);
+            case 16: return launch_pair<0, 16>(amap, bmap, sfamap, sfbmap, ymap, gb, replica_boxes, so, fb, pairs, st);
+            case 32: return launch_pair<0, 32>(amap, bmap, sfamap, sfbmap, ymap, gb, replica_boxes, so, fb, pairs, st);
+            case 64: return launch_pair<0, 64>(amap, bmap, sfamap, sfbmap, ymap, gb, replica_boxes, so, fb, pairs, st);
+            case 128: return launch_pair<0, 128>(amap, bmap, sfamap, sfbmap, ymap, gb, replica_boxes, so, fb, pairs, st);
             default: return MACAQ_ERR_UNSUPPORTED;
         }
     }
@@ -590,7 +598,7 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
     const bool grouped = offsets != nullptr;
     const bool pair = !grouped && BN == 256 && rows > 128 && K % 256 == 0;  // 2-SM pairs, 256 x 256 tiles
     const int32_t experts = grouped ? E : 1;
-    GemmArgs g;
+    GemmArgs g{};
     g.asf = Asf;
     g.bsf = Wsf;
     g.y = Y;
@@ -690,7 +698,7 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
     }
     // large M on 2-SM pairs: the ready counts, the work counter and the exit counter fit the region
     f.in_pair = E == 0 && M > kSkinnyMaxM && N % 256 == 0 && K % 256 == 0 &&
-                static_cast<size_t>((M + 127) / 128) * (K / 256) + 2 <= kCountRegion / 4;
+                static_cast<size_t>((M + 127) / 128) * (K / 256 + 1) + 2 <= kCountRegion / 4;
     // the activations never overlap the counter region, whichever kernel runs afterwards
     f.a_off = std::max(f.gemm_ws, up(kCountRegion));
     f.sf_off = f.a_off + up(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
@@ -702,10 +710,11 @@ FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, int32_t E, int sms) {
 // skinny kernel with its quantizer warps: no quantized activation touches HBM. Every other shape (and
 // every grouped call) quantizes X into the workspace and runs the GEMM on it, two launches in stream
 // order: re-quantizing an A tile for every output tile it meets would cost more than the
-// 0.53125 B/element round trip once M is large.
+// 0.53125 B/element round trip once M is large. one_launch: dense M > 128 with N, K % 256 == 0 runs
+// the 2-SM GEMM that quantizes X itself (one launch, ready counts in the counter region).
 macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const int32_t *offsets, int32_t E, int64_t M,
                           int64_t N, int64_t K, const uint8_t *Wq, const uint8_t *Wsf, void *Y, int32_t out_dtype,
-                          void *workspace, size_t ws_bytes, cudaStream_t st) {
+                          void *workspace, size_t ws_bytes, cudaStream_t st, bool one_launch = false) {
     if (M < 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 128 != 0) return MACAQ_ERR_SHAPE;
     if (!valid_block(b)) return MACAQ_ERR_UNSUPPORTED;
     if (offsets != nullptr && (E < 1 || E > 1024)) return MACAQ_ERR_SHAPE;
@@ -723,7 +732,7 @@ macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const in
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if (offsets == nullptr && f.in_kernel)
         return run_skinny(X, nullptr, inv_s, b, M, N, K, Wq, Wsf, Y, out_dtype, ws, f.gemm_ws, dev.sms, st);
-    if (offsets == nullptr && f.in_pair) {
+    if (one_launch && offsets == nullptr && f.in_pair) {
         // one launch: the 2-SM GEMM quantizes X into the workspace itself (ready counts in the
         // counter region) and reads A from there
         FusedA fa{};
@@ -736,7 +745,8 @@ macaq_status linear_fused(const void *X, const float *inv_s, int32_t b, const in
         fa.units = fa.rt_count * fa.kb_count * kFaUnitsPerBlock;
         int32_t *counters = reinterpret_cast<int32_t *>(ws);
         fa.flags = counters;
-        fa.next_unit = counters + fa.rt_count * fa.kb_count;
+        fa.rt_done = counters + fa.rt_count * fa.kb_count;
+        fa.next_unit = fa.rt_done + fa.rt_count;
         fa.exit_count = fa.next_unit + 1;
         GemmArgs g{};
         g.asf = ws + f.sf_off;
@@ -1129,9 +1139,9 @@ macaq_status macaq_moe_combine(const void *Y, int64_t y_rows, int64_t N, const i
 macaq_status macaq_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s, int64_t M, int64_t N,
                           int64_t K, int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
                           int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
-    if (mode == MACAQ_A_BF16_FUSED)
+    if (mode == MACAQ_A_BF16_FUSED || mode == MACAQ_A_BF16_ONE_LAUNCH)
         return macaq::linear_fused(A, inv_s, had_block, nullptr, 0, M, N, K, Wq, Wsf, Y, out_dtype, workspace, ws_bytes,
-                                   static_cast<cudaStream_t>(stream));
+                                   static_cast<cudaStream_t>(stream), mode == MACAQ_A_BF16_ONE_LAUNCH);
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
     return macaq::gemm(static_cast<const uint8_t *>(A), Asf, nullptr, 1, M, N, K, Wq, Wsf, Y, out_dtype, workspace,
                        ws_bytes, static_cast<cudaStream_t>(stream));
@@ -1141,7 +1151,7 @@ macaq_status macaq_linear_fixed_scratch(int32_t mode, const void *A, const uint8
                                         int64_t M, int64_t N, int64_t K, int32_t had_block, const uint8_t *Wq,
                                         const uint8_t *Wsf, void *Y, int32_t out_dtype, macaq_stream_t stream) {
     (void)inv_s, (void)had_block;
-    if (mode == MACAQ_A_BF16_FUSED) return MACAQ_ERR_UNSUPPORTED;
+    if (mode == MACAQ_A_BF16_FUSED || mode == MACAQ_A_BF16_ONE_LAUNCH) return MACAQ_ERR_UNSUPPORTED;
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
     return macaq::linear_fixed_scratch(static_cast<const uint8_t *>(A), Asf, M, N, K, Wq, Wsf, Y, out_dtype,
                                        static_cast<cudaStream_t>(stream));
@@ -1152,7 +1162,7 @@ macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *As
                                   int32_t had_block, const uint8_t *Wq, const uint8_t *Wsf, void *Y,
                                   int32_t out_dtype, void *workspace, size_t ws_bytes, macaq_stream_t stream) {
     if (group_offsets == nullptr) return MACAQ_ERR_INVALID_ARG;
-    if (mode == MACAQ_A_BF16_FUSED)
+    if (mode == MACAQ_A_BF16_FUSED || mode == MACAQ_A_BF16_ONE_LAUNCH)
         return macaq::linear_fused(A, inv_s, had_block, group_offsets, E, total_rows, N, K, Wq, Wsf, Y, out_dtype,
                                    workspace, ws_bytes, static_cast<cudaStream_t>(stream));
     if (mode != MACAQ_A_QUANTIZED) return MACAQ_ERR_INVALID_ARG;
