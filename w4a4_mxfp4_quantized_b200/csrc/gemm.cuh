@@ -906,8 +906,9 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
 // 128x256b copy each per K-block. The stage ring has up to kSkinnyMaxStages stages; the accumulator
 // is double-buffered in TMEM. Needs K % 256 == 0.
 //
-// Fused form (kFusedB = Hadamard block b > 0, M <= 16; the library uses it for M <= 4, where it is
-// faster than a separate quantizer launch): the activations arrive as bf16 X. Per stage
+// Fused form (kFusedB = Hadamard block b > 0; dispatched, and tested, for M <= kSkinnyFusedMaxM = 4
+// only, where it is faster than a separate quantizer launch; the host also requires a stage count
+// divisible by four, so each quantizer warp owns whole stages): the activations arrive as bf16 X. Per stage
 // the producer also loads X's K-block (16 rows x 256 bf16 by TMA, zero-filled past M) and the
 // K-block's 256 multipliers 1/s (bulk copy); four quantizer warps (warps 6-9, one 32-element group
 // per thread: row t / 8, group t % 8) apply scale, Hadamard and MXFP4 exactly as the quantizer kernel

@@ -397,7 +397,7 @@ SkinnyPlan skinny_plan_cached(int64_t M, int64_t N, int64_t K, int sms, bool fus
 }
 
 // The skinny GEMM. fused_b = 0: A is Xq/Asf (quantized activations). fused_b > 0: A is bf16 X
-// (M <= 16) and the kernel applies 1/s (inv_s, may be null), H_b and MXFP4 itself.
+// (M <= kSkinnyFusedMaxM) and the kernel applies 1/s (inv_s, may be null), H_b and MXFP4 itself.
 template <int kFusedB>
 macaq_status launch_skinny(const CUtensorMap &wmap, const CUtensorMap &xmap, const CUtensorMap &sfwmap,
                            const CUtensorMap &sfxmap, const CUtensorMap &ymap, const SkinnyArgs &g, const SkinnyPlan &p,
@@ -421,6 +421,7 @@ macaq_status run_skinny(const void *A, const uint8_t *Asf, const float *inv_s, i
     // the in-kernel quantizer warps take the stages in turn, four at a time: a stage count that is
     // not a multiple of four would give one stage to two warps at different phases
     if (fused && p.stages % 4 != 0) return MACAQ_ERR_UNSUPPORTED;
+    if (fused && M > kSkinnyFusedMaxM) return MACAQ_ERR_SHAPE;   // the only sizes it is tested for
     if (ws_bytes < p.partial_bytes + p.count_bytes) return MACAQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MACAQ_ERR_ALIGNMENT;
     CUtensorMap wmap, xmap, sfwmap, sfxmap, ymap;

@@ -167,10 +167,10 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&raw)[4], uint64_t (
 // one 32-bit store in the tiled layout. e < 0 marks a row outside every group: nothing is stored.
 // The whole warp calls it together (shuffles).
 template <int kB, bool kWeight>
-__device__ __forceinline__ void quantize_store_group(uint64_t (&p)[16], const uint64_t (&mv)[16], const QuantArgs &a,
-                                                     int e, uint32_t m, uint32_t g, const int32_t *s_off,
-                                                     const int32_t *s_tb, int lane) {
-    if (a.mul != nullptr) {
+__device__ __forceinline__ void quantize_store_group(uint64_t (&p)[16], const uint64_t (&mv)[16], bool with_mul,
+                                                     const QuantArgs &a, int e, uint32_t m, uint32_t g,
+                                                     const int32_t *s_off, const int32_t *s_tb, int lane) {
+    if (with_mul) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
     }
@@ -192,9 +192,9 @@ __device__ __forceinline__ void quantize_store_group(uint64_t (&p)[16], const ui
 // stages (activations: no 1/b), then each value rounded to bf16 (nearest even); the 64 bytes go to
 // row m, group g of a bf16 [rows, K] output (a.q reinterpreted). The whole warp calls it (shuffles).
 template <int kB>
-__device__ __forceinline__ void transform_store_bf16_group(uint64_t (&p)[16], const uint64_t (&mv)[16], const QuantArgs &a,
-                                                           bool store, uint32_t m, uint32_t g) {
-    if (a.mul != nullptr) {
+__device__ __forceinline__ void transform_store_bf16_group(uint64_t (&p)[16], const uint64_t (&mv)[16], bool with_mul,
+                                                           const QuantArgs &a, bool store, uint32_t m, uint32_t g) {
+    if (with_mul) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) p[i] = mul2(p[i], mv[i]);
     }
@@ -218,19 +218,26 @@ __device__ __forceinline__ void transform_store_bf16_group(uint64_t (&p)[16], co
     }
 }
 
-// Zeroes the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1): groups are
-// dealt to the CTAs in turn, one warp per padding row, lanes over the 32-bit words (4 scale columns
-// each) of that row.
+// Zeroes the scale factors of every group's padding rows (rows M_e .. 128 * tiles_e - 1, all in the
+// group's last 128-row tile). Work items are (group, 128x4 scale tile of that last row tile), dealt to
+// the warps of all CTAs; a warp writes the tile's 128 words with four coalesced 128-byte stores, each
+// lane zeroing its word only when the word's row is a padding row (word w holds row
+// (w % 4) * 32 + w / 4), so the words of valid rows are never touched.
 __device__ __forceinline__ void zero_sf_padding(const QuantArgs &a, const int32_t *s_off, const int32_t *s_tb, int warp,
                                                 int lane, int warps) {
     const uint32_t kq = a.kg >> 2;
-    for (int e = blockIdx.x; e < a.E; e += gridDim.x) {
+    const uint32_t items = static_cast<uint32_t>(a.E) * kq;
+    for (uint32_t it = blockIdx.x * warps + warp; it < items; it += gridDim.x * warps) {
+        const uint32_t e = it / kq, ct = it - e * kq;
         const uint32_t me = static_cast<uint32_t>(s_off[e + 1] - s_off[e]);
         const uint32_t nt = static_cast<uint32_t>(s_tb[e + 1] - s_tb[e]);
-        for (uint32_t pr = me + warp; pr < nt * 128; pr += warps) {
-            const uint32_t sf_row = static_cast<uint32_t>(s_tb[e]) * 128 + pr;
-            for (uint32_t w = lane; w < kq; w += 32)
-                *reinterpret_cast<uint32_t *>(a.sf + sf_offset(sf_row, 4 * w, kq)) = 0u;
+        if (nt == 0 || me == nt * 128) continue;
+        const uint32_t first = (nt - 1) * 128;   // the last tile's first row, counted inside the group
+        uint32_t *tile = reinterpret_cast<uint32_t *>(a.sf + sf_offset((static_cast<uint32_t>(s_tb[e]) + nt - 1) * 128, 4 * ct, kq));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t w = j * 32 + lane;
+            if (first + (w & 3) * 32 + (w >> 2) >= me) tile[w] = 0u;
         }
     }
 }
@@ -268,7 +275,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
         fence_mbar_init();
         if (rt_begin < rt_end) prefetch_tensor_map(&xmap);
     }
-    griddep_wait();  // X, the offsets and the outputs may belong to the previous kernel in the stream
+    griddep_wait();  // X, the multipliers, the offsets and the outputs may belong to the previous kernel
     load_group_layout(a.offsets, a.E, a.rows, s_off, s_tb);  // contains __syncthreads
     griddep_launch_dependents();
 
@@ -323,8 +330,8 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[s]);
-            if constexpr (kBf16Out) transform_store_bf16_group<kB>(p, mv, a, e >= 0, m, g);
-            else quantize_store_group<kB, kWeight>(p, mv, a, e, m, g, s_off, s_tb, lane);
+            if constexpr (kBf16Out) transform_store_bf16_group<kB>(p, mv, a.mul != nullptr, a, e >= 0, m, g);
+            else quantize_store_group<kB, kWeight>(p, mv, a.mul != nullptr, a, e, m, g, s_off, s_tb, lane);
         }
     }
 
@@ -407,7 +414,7 @@ __global__ void __launch_bounds__(kQConsumers, 2) quant_gather_kernel(QuantArgs 
         }
         uint64_t p[16];
         unpack_bf16x32(raw, p);
-        quantize_store_group<kB, false>(p, mv, a, e, m, g, s_off, s_tb, lane);
+        quantize_store_group<kB, false>(p, mv, a.mul != nullptr, a, e, m, g, s_off, s_tb, lane);
     }
     zero_sf_padding(a, s_off, s_tb, warp, lane, kQConsumers / 32);
 }
