@@ -732,44 +732,42 @@ def _r(x, n=3):
 
 
 def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None):
-    """Short strings of the sections, so that the whole line stays a few KB."""
-    out = {}
+    """Short strings of the sections (the full numbers go to --details), so that the whole line stays
+    about 3 KB. Legend: g = GEMM alone, aq = act_quant alone, f = one-call layer, wo = weight-only
+    layer (us); fp4 / hbm = fraction of the FP4 / HBM peak; B = transform pipeline vs plain MXFP4,
+    1L = the one-launch form vs plain MXFP4; fusedW = Qwen3 layer with fused QKV and GateUp weights;
+    sw = gate/up GEMM with the SwiGLU epilogue vs the two-step form (us)."""
+    out = {"legend": "us; g gemm, aq act_quant, f one-call layer, wo weight-only, B vs plain mxfp4, 1L one launch"}
     if sweep:
         out["sweep"] = " | ".join(
-            f"M{p['M']}: gemm {p['gemm_us']:.1f}us {p['gemm_frac_hbm']:.2f}hbm {p['gemm_frac_fp4_peak']:.2f}fp4, "
-            f"aq {p['act_quant_us']:.1f}us, fused {p['fused_layer_us']:.1f}us"
-            + (f", w4a16 {p['w4a16_layer_us']:.1f}us" if p.get("w4a16_layer_us") else "") for p in sweep)
-    out["overhead"] = {k: _r(overhead[k]) for k in ("B_vs_plain_mxfp4_pipeline", "A_vs_gemm_on_prequantized_A",
-                                                     "two_kernel_B")}
+            f"M{p['M']} g{p['gemm_us']:.1f} {p['gemm_frac_hbm']:.2f}hbm {p['gemm_frac_fp4_peak']:.2f}fp4 "
+            f"aq{p['act_quant_us']:.1f} f{p['fused_layer_us']:.1f}"
+            + (f" wo{p['w4a16_layer_us']:.1f}" if p.get("w4a16_layer_us") else "") for p in sweep)
+    out["overhead"] = {k: _r(overhead[k]) for k in ("B_vs_plain_mxfp4_pipeline", "A_vs_gemm_on_prequantized_A")}
     if prefill:
         out["prefill"] = " | ".join(
-            f"{p['M']}x{p['K']}x{p['N']}: gemm {p['gemm_ms']:.3f}ms {p['gemm_frac_fp4_peak']:.2f}fp4, "
-            f"B {100 * p['overhead_B_transform']:+.1f}% (one launch {100 * p['overhead_B_fused']:+.1f}%) "
-            f"(aq only {100 * p['overhead_B_act_quant_only']:+.1f}%), "
-            f"A {100 * p['overhead_A_transform']:+.1f}%, aq {p['act_quant_frac_hbm']:.2f}hbm" for p in prefill["points"])
+            f"{p['M'] // 1024}k{p['K'] // 1024}k{p['N'] // 1024}k {p['gemm_frac_fp4_peak']:.2f}fp4 "
+            f"B{100 * p['overhead_B_transform']:+.1f}% 1L{100 * p['overhead_B_fused']:+.0f}% "
+            f"aq{p['act_quant_frac_hbm']:.2f}hbm" for p in prefill["points"])
     if qwen3:
         out["qwen3"] = " | ".join(
-            f"M{p['M']}: {p['layer_us']:.0f}us {p['layer_tflops']:.0f}TF {p['layer_frac_hbm']:.2f}hbm "
-            f"{p['layer_frac_fp4_peak']:.2f}fp4, fusedW {p['layer_fused_qkv_gateup_us']:.0f}us, "
-            f"swiglu chain {p['layer_swiglu_chain_us']:.0f}us (gate/up+swiglu {p['swiglu_fused_us']:.0f} vs "
-            f"{p['swiglu_two_step_us']:.0f}us)" for p in qwen3["points"])
+            f"M{p['M']} {p['layer_us']:.0f}us fusedW{p['layer_fused_qkv_gateup_us']:.0f} "
+            f"sw{p['swiglu_fused_us']:.0f}/{p['swiglu_two_step_us']:.0f}" for p in qwen3["points"])
     if moe:
         def glue(p):
-            if "gather_act_quant_us" in p:
-                return f", gather aq {p['gather_act_quant_us']:.1f}us vs {p['grouped_act_quant_us']:.1f}"
             if "combine_us" in p:
-                return f", combine {p['combine_us']:.1f}us {p['combine_frac_hbm']:.2f}hbm"
+                return f" comb{p['combine_frac_hbm']:.2f}hbm"
             return ""
         out["moe"] = " | ".join(
-            f"{p['proj']} T{p['T']}: gemm {p['grouped_gemm_us']:.1f}us {p['grouped_gemm_frac_hbm']:.2f}hbm "
-            f"{p['grouped_gemm_frac_fp4_peak']:.2f}fp4, aq {p['grouped_act_quant_frac_hbm']:.2f}hbm{glue(p)}"
+            f"{'gu' if p['proj'] == 'gate_up' else 'dn'}T{p['T']} g{p['grouped_gemm_us']:.0f} "
+            f"{p['grouped_gemm_frac_hbm']:.2f}hbm {p['grouped_gemm_frac_fp4_peak']:.2f}fp4{glue(p)}"
             for p in moe["points"])
     if flip:
-        out["flip_refine"] = f"{flip['ms']:.1f}ms, {flip['moves_per_row']:.0f} moves/row"
+        out["flip_refine"] = f"{flip['ms']:.0f}ms {flip['moves_per_row']:.0f}moves/row"
     if prep:
         out["weight_prep"] = f"{prep['us']:.1f}us {prep['frac_hbm']:.2f}hbm"
     if ceiling:
-        out["copy_ceiling"] = "; ".join(f"{c['bytes'] / 1e6:.1f}MB copy {c['us']:.1f}us {c['gbs']:.0f}GB/s" for c in ceiling)
+        out["copy_ceiling"] = "; ".join(f"{c['bytes'] / 1e6:.0f}MB {c['gbs']:.0f}GB/s" for c in ceiling)
     return out
 
 
@@ -894,7 +892,7 @@ def main():
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
     out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip)
-    out["summary"]["gemm_alone"] = f"{gemm_ms * 1e3:.1f}us {flops / (gemm_ms * 1e-3) / 1e12 / fp4_peak:.3f}fp4 (pre-quantized A)"
+    out["summary"]["gemm_alone"] = f"{gemm_ms * 1e3:.1f}us {flops / (gemm_ms * 1e-3) / 1e12 / fp4_peak:.3f}fp4"
     if args.details:
         with open(args.details, "w") as f:
             json.dump({**out, "sweep": sweep, "transform_overhead": overhead, "prefill": prefill, "qwen3": qwen3,

@@ -109,6 +109,14 @@ def test_fused_mode_rejects_bad_arguments(lib):
     assert lib.macaq_linear(*args(ws=P + 8)) == 3      # misaligned workspace
     assert lib.macaq_linear(*args(M=0)) == 0           # M == 0: no-op
     assert lib.macaq_linear_fixed_scratch(1, P, None, P, 16, 256, 256, 32, P, P, P, 0, None) == 4
+    # mode 2 = MACAQ_A_BF16_ONE_LAUNCH: the same arguments and checks
+    assert lib.macaq_linear(*args(mode=2, b=3)) == 4
+    assert lib.macaq_linear(*args(mode=2, K=200)) == 2
+    assert lib.macaq_linear(*args(mode=2, A=P + 4)) == 3
+    assert lib.macaq_linear(*args(mode=2, M=0)) == 0
+    assert lib.macaq_linear(*args(mode=3)) == 1        # no such mode
+    assert lib.macaq_linear_fixed_scratch(2, P, None, P, 16, 256, 256, 32, P, P, P, 0, None) == 4
+    assert mq.A_BF16_ONE_LAUNCH == 2
     g = lambda off, E: lib.macaq_grouped_linear(1, P, None, P, off, E, 16, 256, 256, 32, P, P, P, 0, P, 1 << 20, None)
     assert g(None, 4) == 1                             # grouped needs offsets
     assert g(P, 0) == 2                                # E < 1
