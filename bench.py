@@ -607,6 +607,48 @@ def weight_prep_section(dev, hbm, steps=10):
             "gbs": b / (ms * 1e-3) / 1e9, "frac_hbm": b / (ms * 1e-3) / 1e9 / hbm}
 
 
+def had_block_section(dev, hbm, fp4_peak, M=2048, steps=20):
+    """The Llama-3-8B up/gate layer at M = 2048 with each Hadamard block size b in {16, 32, 64, 128}
+    (weights prepared per b): act_quant alone and act_quant + GEMM, timed side by side. Inputs rotate
+    over copies larger than twice L2."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    c = inputs.llama3_8b_up(M, draw_w=True)
+    W, s = c.W.to(dev), c.s.to(dev)
+    ncopy = copies_for(M)
+    X = [c.X.to(dev)] + [None] * (ncopy - 1)
+    for i in range(1, ncopy):
+        X[i] = X[0].clone()
+    Xq = [torch.empty(M, K_DIM // 2, dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+    Xsf = [torch.empty(mq.sf_bytes(M, K_DIM), dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+    Y = [torch.empty(M, N_DIM, dtype=torch.bfloat16, device=dev) for _ in range(ncopy)]
+    flops = 2.0 * M * N_DIM * K_DIM
+    aq_bytes = M * K_DIM * 2.53125
+    out = []
+    for b in (16, 32, 64, 128):
+        Wq, Wsf, inv = mq.prep_weights(W, s, b)
+        Wqs = [Wq] + [Wq.clone() for _ in range(ncopy - 1)]
+        Wsfs = [Wsf] + [Wsf.clone() for _ in range(ncopy - 1)]
+
+        def aq(i, b=b, inv=inv):
+            j = i % ncopy
+            mq.act_quant(X[j], inv, b, Xq=Xq[j], Xsf=Xsf[j])
+
+        def layer(i, b=b, inv=inv, Wqs=Wqs, Wsfs=Wsfs):
+            j = i % ncopy
+            mq.act_quant(X[j], inv, b, Xq=Xq[j], Xsf=Xsf[j])
+            mq.linear(Xq[j], Xsf[j], Wqs[j], Wsfs[j], Y=Y[j])
+
+        t = time_graphs_interleaved({"aq": aq, "layer": layer}, steps, torch.cuda.current_stream(dev))
+        out.append({"had_block": b, "act_quant_us": t["aq"] * 1e3,
+                    "act_quant_frac_hbm": aq_bytes / (t["aq"] * 1e-3) / 1e9 / hbm,
+                    "layer_us": t["layer"] * 1e3, "layer_tflops": flops / (t["layer"] * 1e-3) / 1e12})
+        del Wqs, Wsfs
+    assert mq.device_status() == 0
+    return {"workload": f"llama3_8b_up_gate M={M} K={K_DIM} N={N_DIM}, b in 16..128", "points": out}
+
+
 def profile_mode(M, steps, warmup, dev, form="layer"):
     """Eager layer passes with no timing: the commands the ncu captures run. form: "layer" (act_quant
     then the GEMM), "fused" (the one-call layer from bf16 X), "w4a16" (the weight-only layer)."""
@@ -731,7 +773,7 @@ def _r(x, n=3):
     return None if x is None else float(f"{x:.{n}g}")
 
 
-def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None):
+def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None, hb=None):
     """Short strings of the sections (the full numbers go to --details), so that the whole line stays
     about 3 KB. Legend: g = GEMM alone, aq = act_quant alone, f = one-call layer, wo = weight-only
     layer (us); fp4 / hbm = fraction of the FP4 / HBM peak; B = transform pipeline vs plain MXFP4,
@@ -762,6 +804,9 @@ def summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip=None):
             f"{'gu' if p['proj'] == 'gate_up' else 'dn'}T{p['T']} g{p['grouped_gemm_us']:.0f} "
             f"{p['grouped_gemm_frac_hbm']:.2f}hbm {p['grouped_gemm_frac_fp4_peak']:.2f}fp4{glue(p)}"
             for p in moe["points"])
+    if hb:
+        out["had_block"] = " | ".join(f"b{p['had_block']} aq{p['act_quant_us']:.1f} layer{p['layer_us']:.1f}"
+                                      for p in hb["points"])
     if flip:
         out["flip_refine"] = f"{flip['ms']:.0f}ms {flip['moves_per_row']:.0f}moves/row"
     if prep:
@@ -830,7 +875,7 @@ def main():
     gemm_tflops = flops / ((fused_ms if fused_step else gemm_ms) * 1e-3) / 1e12
     gemm_kernel = gemm_kernel_name(M) + (" (one launch, quantizing X itself)" if fused_step else "")
     aq_bytes = M * K_DIM * (2 + 0.5 + 1 / 32)
-    sweep, prefill, qwen3, moe, prep, ceiling, flip = [], None, None, None, None, [], None
+    sweep, prefill, qwen3, moe, prep, ceiling, flip, hb = [], None, None, None, None, [], None, None
     if not args.no_sweep:
         for m in M_SWEEP:
             tot, aq, gm, Lm = time_layer(m, max(10, args.steps), args.warmup, dev, dist_on, fused=True)
@@ -864,6 +909,7 @@ def main():
         qwen3 = qwen3_section(dev, hbm, fp4_peak)
         moe = moe_section(dev, hbm, fp4_peak)
         prep = weight_prep_section(dev, hbm)
+        hb = had_block_section(dev, hbm, fp4_peak)
         flip = flip_section(dev)
         ceiling = [copy_ceiling(dev, aq_bytes), copy_ceiling(dev, 16384 * 16384 * 2.53125)]
     if rank != 0:
@@ -891,12 +937,13 @@ def main():
         "clocks": dict(clocks, window="warm replays (1.5 s of this workload) and the timed replay"),
     }
     out["cpu_baseline"] = cpu_baseline(M) if world == 1 else None
-    out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip)
+    out["summary"] = summary(sweep, overhead, prefill, qwen3, moe, prep, ceiling, flip, hb)
     out["summary"]["gemm_alone"] = f"{gemm_ms * 1e3:.1f}us {flops / (gemm_ms * 1e-3) / 1e12 / fp4_peak:.3f}fp4"
     if args.details:
         with open(args.details, "w") as f:
             json.dump({**out, "sweep": sweep, "transform_overhead": overhead, "prefill": prefill, "qwen3": qwen3,
-                       "moe": moe, "weight_prep": prep, "copy_ceiling": ceiling, "flip_refine": flip}, f, indent=1)
+                       "moe": moe, "weight_prep": prep, "copy_ceiling": ceiling, "flip_refine": flip,
+                       "had_block": hb}, f, indent=1)
     print(json.dumps(out))
     if dist_on:
         torch.distributed.destroy_process_group()
