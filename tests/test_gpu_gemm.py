@@ -191,12 +191,23 @@ def grouped_tiled_sf(Asf, offsets, K):
     return buf
 
 
+_PAIR_SIZES = [0, 513, 7, 256, 255, 900, 128, 1, 0, 640, 384, 129, 1000, 2, 300, 17, 760, 64, 3, 222]
+
+
 @pytest.mark.parametrize("offsets,N,K", [
     ([0, 5, 5, 140, 141, 141, 300], 256, 256),
     ([0, 0, 1, 129, 257, 257], 128, 384),
     ([0, 64, 64, 64, 200], 512, 1024),
+    # at least 256 rows per expert on average, N and K multiples of 256: the 2-SM grouped form, with
+    # empty experts, one-row experts, odd tile counts (a pair's second half past its expert) and
+    # partial tiles
+    ([0, 0, 300, 429, 1429, 1430, 2130], 512, 512),
+    ([0, 1024, 1024, 2500], 768, 768),
+    ([0] + list(np.cumsum(_PAIR_SIZES)), 256, 1024),
 ])
 def test_grouped_random_codes(offsets, N, K):
+    """Every output of the grouped GEMM against the oracle (fp32 within 1e-5 of sum|terms|, bf16 the
+    rounded fp32), on random codes and scales."""
     E = len(offsets) - 1
     M = offsets[-1]
     Aq, Asf, Wq, Wsf = random_operands(E * 11 + K, M, N, K, E=E)

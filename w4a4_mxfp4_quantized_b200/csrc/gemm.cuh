@@ -187,14 +187,19 @@ __device__ __forceinline__ void store_chunk_tma(const CUtensorMap *ymap, uint8_t
     }
 }
 
+// row_end: rows at or past it are not written (the grouped form's expert bound; dense calls pass a
+// bound past every row and rely on the tensor map's clipping). A warp whose 32 rows all lie below it
+// stores through TMA; a warp that straddles it stores its live rows with plain 16-byte stores.
 __device__ __forceinline__ void epilogue_tile_pair(uint32_t tmem, int warp, int lane, int32_t row0, int32_t col0,
                                                    bool out_f32, const CUtensorMap *ymap, uint8_t *buf,
-                                                   uint32_t accum_empty_addr) {
+                                                   uint32_t accum_empty_addr, int64_t row_end, void *y, int32_t ldy) {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
     const int32_t row = row0 + quarter * 32;
     const int32_t col = col0 + half * 128;
+    const bool whole = static_cast<int64_t>(row) + 32 <= row_end;
+    const bool live = static_cast<int64_t>(row) + lane < row_end;
     if (out_f32) {
         uint32_t v[128];
         tmem_ld64(taddr, *reinterpret_cast<uint32_t(*)[64]>(v));
@@ -203,8 +208,14 @@ __device__ __forceinline__ void epilogue_tile_pair(uint32_t tmem, int warp, int 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+        if (whole) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) store_chunk_tma(ymap, buf, lane, v + 32 * c, col + 32 * c, row);
+            for (int c = 0; c < 4; ++c) store_chunk_tma(ymap, buf, lane, v + 32 * c, col + 32 * c, row);
+        } else if (live) {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<float *>(y) + (static_cast<int64_t>(row) + lane) * ldy + col);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) dst[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        }
     } else {
         uint32_t packed[64];
 #pragma unroll
@@ -221,8 +232,15 @@ __device__ __forceinline__ void epilogue_tile_pair(uint32_t tmem, int warp, int 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(accum_empty_addr);
+        if (whole) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) store_chunk_tma(ymap, buf, lane, packed + 32 * c, col + 64 * c, row);
+            for (int c = 0; c < 2; ++c) store_chunk_tma(ymap, buf, lane, packed + 32 * c, col + 64 * c, row);
+        } else if (live) {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(y) + (static_cast<int64_t>(row) + lane) * ldy + col);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        }
     }
 }
 
@@ -633,7 +651,7 @@ __device__ __forceinline__ void epilogue_tile_pair_swiglu(uint32_t tmem, int war
     store_swiglu64(o, static_cast<int64_t>(row0) + quarter * 32 + lane, M, c0, codes, E8);
 }
 
-template <int kSwiglu, int kFusedB = 0>
+template <int kSwiglu, int kFusedB = 0, bool kGrouped = false>
 __global__ void __launch_bounds__(PairCfg::kThreads, 1)
 gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                       const __grid_constant__ CUtensorMap sfamap, const __grid_constant__ CUtensorMap sfbmap,
@@ -654,6 +672,11 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     uint8_t *sB = sA + S * C::kABytes;
     uint8_t *sSfx = sB + S * C::kBBytes;
     uint8_t *sEpi = sSfx + S * C::kSfxBytes;
+    // grouped form: the expert row offsets, the first 128-row tile of each expert and the first
+    // 256-row pair tile of each expert (each [E + 1]), after the epilogue buffers
+    int32_t *s_off = reinterpret_cast<int32_t *>(sEpi + C::kEpiBytes);
+    int32_t *s_tb = s_off + (g.E + 1);
+    int32_t *s_pb = s_tb + (g.E + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -661,9 +684,10 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     const bool leader = rank == 0;
     const uint32_t cluster = blockIdx.x >> 1;
     const uint32_t clusters = gridDim.x >> 1;
-    const uint32_t m_tiles = static_cast<uint32_t>((g.rows + 255) / 256);
+    // dense: the host launches at most num_tiles pairs; grouped: the tile count is read on the device
+    uint32_t m_tiles = static_cast<uint32_t>((g.rows + 255) / 256);
     const uint32_t n_tiles = static_cast<uint32_t>(g.N / 256);
-    const uint32_t num_tiles = m_tiles * n_tiles;  // the host launches at most this many pairs
+    uint32_t num_tiles = m_tiles * n_tiles;
     const uint32_t band_m = g.raster_m > 0 ? static_cast<uint32_t>(g.raster_m) : static_cast<uint32_t>(kRasterM);
     const int K = g.K;
     const int kq = K / 128;
@@ -702,6 +726,43 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
     tc_fence_after();
     griddep_wait();  // the operands and Y may belong to the previous kernel in the stream
     griddep_launch_dependents();
+    if constexpr (kGrouped) {
+        // pair tiles: expert e has ceil(tiles_e / 2) of them; s_pb is their exclusive prefix. Both CTAs
+        // of a pair read the same offsets, so they walk the same tiles.
+        load_group_layout(g.offsets, g.E, g.rows, s_off, s_tb);   // contains __syncthreads
+        if (warp == 0) {
+            int32_t carry = 0;
+            for (int base = 0; base <= g.E; base += 32) {
+                const int e = base + lane;
+                int32_t x = (e > 0 && e <= g.E) ? (s_tb[e] - s_tb[e - 1] + 1) / 2 : 0;   // pair tiles of expert e - 1
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int32_t y = __shfl_up_sync(0xffffffffu, x, d);
+                    if (lane >= d) x += y;
+                }
+                if (e <= g.E) s_pb[e] = carry + x;
+                carry += __shfl_sync(0xffffffffu, x, 31);
+            }
+        }
+        __syncthreads();
+        m_tiles = static_cast<uint32_t>(s_pb[g.E]);
+        num_tiles = m_tiles * n_tiles;
+    }
+    // grouped: pair-row tile mt -> its expert, this CTA's 128-row tile inside the SF layout (rt), its
+    // first row and the expert's row bound (row_end <= row0 when this half lies past the expert)
+    auto pair_rows = [&](uint32_t mt, int &expert, int32_t &rt, int64_t &row0, int64_t &row_end) {
+        int lo = 0, hi = g.E;   // s_pb[lo] <= mt < s_pb[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (static_cast<uint32_t>(s_pb[mid]) <= mt) lo = mid;
+            else hi = mid;
+        }
+        expert = lo;
+        const int32_t local = static_cast<int32_t>(mt - static_cast<uint32_t>(s_pb[lo])) * 2 + static_cast<int32_t>(rank);
+        rt = s_tb[lo] + local;
+        row0 = s_off[lo] + static_cast<int64_t>(local) * 128;
+        row_end = min(static_cast<int64_t>(s_off[lo + 1]), row0 + 128);
+    };
     const uint32_t tmem = tmem_slot;
     const uint32_t leader_failed_addr = map_to_rank(smem_u32(const_cast<int *>(&failed)), 0);
 
@@ -717,10 +778,21 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
             for (uint32_t sgi = 0; !stop && segment(sgi, t, k0, k1); ++sgi) {
                 uint32_t mt, nt;
                 raster(t, m_tiles, n_tiles, band_m, mt, nt);
-                const int32_t arow = static_cast<int32_t>(mt * 256 + rank * 128);
-                const int32_t brow = static_cast<int32_t>(nt * 256 + rank * 128);
-                const int32_t a_tile = static_cast<int32_t>((mt * 2 + rank) * kq);   // first 128x4 tile of A's rows
-                const int32_t b_tile = static_cast<int32_t>(nt * 2 * kq);            // of B's first 128 rows
+                int32_t arow = static_cast<int32_t>(mt * 256 + rank * 128);
+                int32_t brow = static_cast<int32_t>(nt * 256 + rank * 128);
+                int32_t a_tile = static_cast<int32_t>((mt * 2 + rank) * kq);   // first 128x4 tile of A's rows
+                int32_t b_tile = static_cast<int32_t>(nt * 2 * kq);            // of B's first 128 rows
+                if constexpr (kGrouped) {
+                    // a half past its expert loads whatever rows and scales lie there (zeros past the
+                    // tensors); the epilogue writes none of its rows
+                    int expert, rt;
+                    int64_t row0, row_end;
+                    pair_rows(mt, expert, rt, row0, row_end);
+                    arow = static_cast<int32_t>(row0);
+                    a_tile = rt * kq;
+                    brow = expert * g.N + static_cast<int32_t>(nt * 256 + rank * 128);
+                    b_tile = (expert * (g.N / 128) + static_cast<int32_t>(nt * 2)) * kq;
+                }
                 // fused form: once the row tile's units have all finished, its K-blocks need no checks;
                 // otherwise a_ready_end is the end of the run of K-blocks known to be finished
                 int a_ready_end = num_kb;
@@ -843,6 +915,11 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
         for (uint32_t sgi = 0; segment(sgi, t, k0, k1); ++sgi, ++tiles_done) {
             uint32_t mt, nt;
             raster(t, m_tiles, n_tiles, band_m, mt, nt);
+            int64_t row0 = static_cast<int64_t>(mt) * 256 + rank * 128, row_end = int64_t(1) << 62;   // dense: TMA clips at M
+            if constexpr (kGrouped) {
+                int expert, rt;
+                pair_rows(mt, expert, rt, row0, row_end);
+            }
             if constexpr (kFusedB > 0) {
                 // test_wait, not try_wait: a blocking poll would hold the warp for the suspend limit
                 // between units while the accumulator is far from ready
@@ -857,8 +934,8 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_con
                 epilogue_tile_pair_swiglu<kSwiglu>(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128),
                                                    static_cast<int32_t>(nt), g.rows, so, empty_addr);
             else
-                epilogue_tile_pair(tmem, warp, lane, static_cast<int32_t>(mt * 256 + rank * 128), static_cast<int32_t>(nt * 256),
-                                   g.out_f32 != 0, &ymap, sEpi + (warp - 2) * 4096, empty_addr);
+                epilogue_tile_pair(tmem, warp, lane, static_cast<int32_t>(row0), static_cast<int32_t>(nt * 256),
+                                   g.out_f32 != 0, &ymap, sEpi + (warp - 2) * 4096, empty_addr, row_end, g.y, g.N);
         }
         while (units_left && !failed) take_unit();   // units other pairs still wait for
         if (lane == 0) bulk_wait_read();  // shared memory stays valid until this warp's stores have read it

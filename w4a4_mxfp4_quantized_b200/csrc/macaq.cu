@@ -490,11 +490,14 @@ template <int kSwiglu, int kFusedB = 0>
 macaq_status launch_pair(const CUtensorMap &amap, const CUtensorMap &bmap, const CUtensorMap &sfamap,
                          const CUtensorMap &sfbmap, const CUtensorMap &ymap, const GemmArgs &g, int replica_boxes,
                          const SwigluOut &so, const FusedA &fa, unsigned pairs, cudaStream_t st) {
-    auto k = gemm_mxf4_pair_kernel<kSwiglu, kFusedB>;
-    macaq_status s = set_smem(k, PairCfg::kSmemBytes);
+    constexpr bool kGrouped = kSwiglu < 0;   // kSwiglu = -1 selects the grouped form
+    auto k = gemm_mxf4_pair_kernel<kGrouped ? 0 : kSwiglu, kFusedB, kGrouped>;
+    // the grouped form keeps three [E + 1] arrays of the expert layout after the epilogue buffers
+    const size_t smem = PairCfg::kSmemBytes + (kGrouped ? 3 * sizeof(int32_t) * (g.E + 1) : 0);
+    macaq_status s = set_smem(k, smem);
     if (s != MACAQ_OK) return s;
-    return launch(k, dim3(2 * pairs), dim3(PairCfg::kThreads), PairCfg::kSmemBytes, st, 2, amap, bmap, sfamap, sfbmap,
-                  ymap, g, replica_boxes, so, fa);
+    return launch(k, dim3(2 * pairs), dim3(PairCfg::kThreads), smem, st, 2, amap, bmap, sfamap, sfbmap, ymap, g,
+                  replica_boxes, so, fa);
 }
 
 // fused_b > 0: A and Asf are the workspace buffers that the kernel itself fills from fa.x (the fused
@@ -503,11 +506,17 @@ macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_
                       const uint8_t *Wsf, void *Y, int32_t out_dtype, const GemmArgs &g, int32_t swiglu_b,
                       const SwigluOut &so, int sms, cudaStream_t st, int32_t fused_b = 0, const FusedA &fa = FusedA{}) {
     macaq_status s;
+    // grouped form (g.offsets set): W is E stacked [N, K/2] blocks with their SF one after another,
+    // and A's SF starts each expert on a fresh 128-row tile
+    const bool grouped = g.offsets != nullptr;
+    const int64_t experts = grouped ? g.E : 1;
+    const uint64_t sfa_bytes = grouped ? macaq_grouped_sf_bytes(rows, g.E, K) : macaq_sf_bytes(rows, K);
+    const uint64_t sfb_bytes = static_cast<uint64_t>(experts) * macaq_sf_bytes(N, K);
     CUtensorMap amap, bmap, sfamap, sfbmap;
     s = tensor_map_2d(&amap, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kBKBytes, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (s == MACAQ_OK)
-        s = tensor_map_2d(&bmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kBKBytes, 128,
+        s = tensor_map_2d(&bmap, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, experts * N, K / 2, kBKBytes, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     // replica views of the SF buffers: (128 B, half h, 8-row group i, 128x4 tile c); for A the
     // halves are the K-block's two tiles (512 B apart), for B the two 128-row tiles of the
@@ -517,17 +526,17 @@ macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_
     // refuses that view, four 1 KB boxes (one replica each) are used instead
     int replica_boxes = 1;
     if (s == MACAQ_OK) {
-        const uint64_t da[5] = {128, 2, 4, 4, macaq_sf_bytes(rows, K) / 512};
+        const uint64_t da[5] = {128, 2, 4, 4, sfa_bytes / 512};
         const uint64_t sa[4] = {512, 128, 0, 512};
-        const uint64_t db[5] = {128, 2, 4, 4, macaq_sf_bytes(N, K) / 512};
+        const uint64_t db[5] = {128, 2, 4, 4, sfb_bytes / 512};
         const uint64_t sb[4] = {kq * 512, 128, 0, 512};
         const uint32_t box[5] = {128, 2, 4, 4, 1};
         if (tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, da, sa, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK ||
             tensor_map(&sfbmap, Wsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, db, sb, box, CU_TENSOR_MAP_SWIZZLE_NONE) != MACAQ_OK) {
             replica_boxes = 4;
-            const uint64_t da4[4] = {128, 2, 4, macaq_sf_bytes(rows, K) / 512};
+            const uint64_t da4[4] = {128, 2, 4, sfa_bytes / 512};
             const uint64_t sa4[3] = {512, 128, 512};
-            const uint64_t db4[4] = {128, 2, 4, macaq_sf_bytes(N, K) / 512};
+            const uint64_t db4[4] = {128, 2, 4, sfb_bytes / 512};
             const uint64_t sb4[3] = {kq * 512, 128, 512};
             const uint32_t box4[4] = {128, 2, 4, 1};
             s = tensor_map(&sfamap, Asf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, da4, sa4, box4, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -543,9 +552,11 @@ macaq_status run_pair(const uint8_t *A, const uint8_t *Asf, int64_t rows, int64_
                           N * (f32 ? 4 : 2), f32 ? 32 : 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (s != MACAQ_OK) return s;
-    const int64_t tiles = ((rows + 255) / 256) * (N / 256);
+    // grouped: the tile count is known on the device only; sum ceil(tiles_e / 2) <= rows / 256 + E
+    const int64_t tiles = ((rows + 255) / 256 + (grouped ? experts : 0)) * (N / 256);
     const int64_t max_pairs = sms / 2;
     const unsigned pairs = static_cast<unsigned>(tiles < max_pairs ? tiles : max_pairs);
+    if (grouped) return launch_pair<-1>(amap, bmap, sfamap, sfbmap, ymap, g, replica_boxes, so, fa, pairs, st);
     if (fused_b > 0) {
         // in-GEMM quantization: raster bands of about two rounds of tiles, so the first round needs
         // only the first band's rows of A; the units follow the same bands
@@ -597,7 +608,10 @@ macaq_status gemm(const uint8_t *A, const uint8_t *Asf, const int32_t *offsets, 
 
     const int BN = (N % 256 == 0) ? 256 : 128;
     const bool grouped = offsets != nullptr;
-    const bool pair = !grouped && BN == 256 && rows > 128 && K % 256 == 0;  // 2-SM pairs, 256 x 256 tiles
+    // 2-SM pairs, 256 x 256 tiles: dense calls with more than 128 rows, grouped calls whose experts
+    // average at least 256 rows (fewer rows per expert leave too many half-empty pairs)
+    const bool pair = BN == 256 && K % 256 == 0 &&
+                      (grouped ? (E <= 1024 && rows >= 256 * static_cast<int64_t>(E)) : rows > 128);
     const int32_t experts = grouped ? E : 1;
     GemmArgs g{};
     g.asf = Asf;
