@@ -354,6 +354,9 @@ macaq_status macaq_swiglu_act_quant(const float *GU, int64_t M, int64_t I, const
  *   Wq             device u8 [E, N, K/2];  Wsf device u8 [E, macaq_sf_bytes(N, K)]
  *   Y              device [total_rows, N] (written; only rows of some expert are written)
  *   workspace      quantized mode: unused (may be NULL); fused mode: as above
+ * With N and K multiples of 256 and total_rows >= 256 * E (experts averaging at least 256 rows) the
+ * GEMM runs on 2-SM pairs (tiles of 256 rows of one expert); otherwise one CTA per 128-row tile.
+ * MACAQ_A_BF16_ONE_LAUNCH is accepted and behaves as MACAQ_A_BF16_FUSED.
  * Source: glonce.com page, paragraph 5 (W4A4 grouped matmul).
  */
 macaq_status macaq_grouped_linear(int32_t mode, const void *A, const uint8_t *Asf, const float *inv_s,
