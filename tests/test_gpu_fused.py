@@ -102,8 +102,12 @@ def test_llama3_8b_up_decode_fused(M):
     check_against_oracle(c, 32, True, Wq, Wsf, y32, rows=np.unique([0, M - 1]))
 
 
-def test_grouped_fused_equals_two_pass():
-    m = inputs.moe_30b_a3b(64, "gate_up")
+@pytest.mark.parametrize("T,mode", [(64, mq.A_BF16_FUSED), (8192, mq.A_BF16_FUSED), (8192, mq.A_BF16_ONE_LAUNCH)])
+def test_grouped_fused_equals_two_pass(T, mode):
+    """The grouped fused call equals the grouped quantizer followed by the grouped GEMM bit for bit;
+    at T = 8192 (512 rows per expert on average) the GEMM runs on 2-SM pairs. The one-launch mode
+    behaves as the fused mode for grouped calls."""
+    m = inputs.moe_30b_a3b(T, "gate_up")
     E = m.offsets.numel() - 1
     K = m.X.shape[1]
     W = m.W.cuda()
@@ -116,12 +120,14 @@ def test_grouped_fused_equals_two_pass():
     X, off = m.X.cuda(), m.offsets.cuda()
     Xq, Xsf = mq.act_quant(X, inv, 32, group_offsets=off)
     ref = mq.grouped_linear(Xq, Xsf, off, Wq, Wsf, out_dtype=mq.OUT_F32)
-    got = mq.grouped_linear(X, None, off, Wq, Wsf, mode=mq.A_BF16_FUSED, inv_s=inv, had_block=32,
-                            out_dtype=mq.OUT_F32)
+    got = mq.grouped_linear(X, None, off, Wq, Wsf, mode=mode, inv_s=inv, had_block=32, out_dtype=mq.OUT_F32)
     torch.cuda.synchronize()
+    assert mq.device_status() == 0
     rows = np.arange(int(m.offsets[-1]))
     assert torch.equal(got[rows].view(torch.int32), ref[rows].view(torch.int32))
     assert counters_zero()
+    if T != 64:
+        return
     # a split-tile skinny call on the same workspace right after the grouped fused call
     c, Wq1, Wsf1, inv1 = layer(31, 64, 1024, 5120, 32, True)
     X1 = c.X.cuda()

@@ -376,7 +376,7 @@ def grouped_linear(A: torch.Tensor, Asf: torch.Tensor | None, group_offsets: tor
     M = A.shape[0]
     dev = A.device
     Y = _out(M, N, out_dtype, dev, Y)
-    fused = mode == A_BF16_FUSED
+    fused = mode in (A_BF16_FUSED, A_BF16_ONE_LAUNCH)
     ws_need = fused_workspace_bytes(M, N, K, E) if fused else workspace_bytes(M, N, K, E)
     if workspace is None and ws_need > 0:
         workspace = _workspace(dev, ws_need)
