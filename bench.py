@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--M", type=int, default=M_MAIN)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--profile", action="store_true", help="eager passes only, for ncu captures")
-    p.add_argument("--profile-form", default="layer", choices=["layer", "fused", "w4a16"])
+    p.add_argument("--profile-form", default="layer", choices=["layer", "fused", "w4a16", "moe"])
     p.add_argument("--details", default=None, help="also write every section's numbers to this JSON file")
     return p.parse_args()
 
@@ -649,11 +649,39 @@ def had_block_section(dev, hbm, fp4_peak, M=2048, steps=20):
     return {"workload": f"llama3_8b_up_gate M={M} K={K_DIM} N={N_DIM}, b in 16..128", "points": out}
 
 
+def profile_moe(steps, warmup, dev, T=8192):
+    """Eager passes of the MoE 30B-A3B gate/up projection at T tokens (grouped act_quant then the
+    grouped GEMM, which runs on 2-SM pairs at T = 8192), for ncu captures."""
+    import w4a4_mxfp4_quantized_b200 as mq
+    from w4a4_mxfp4_quantized_b200 import inputs
+
+    c = inputs.moe_30b_a3b(T, "gate_up")
+    E, N, K = c.W.shape
+    Wq = torch.empty(E, N, K // 2, dtype=torch.uint8, device=dev)
+    Wsf = torch.empty(E, mq.sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    inv = torch.empty(E, K, dtype=torch.float32, device=dev)
+    W, s = c.W.to(dev), c.s.to(dev)
+    for e in range(E):
+        mq.prep_weights(W[e], s[e], HAD_BLOCK, Wq=Wq[e], Wsf=Wsf[e], inv_s=inv[e])
+    del W
+    off = c.offsets.to(dev)
+    X = c.X.to(dev)
+    for _ in range(warmup + steps):
+        Xq, Xsf = mq.act_quant(X, inv, HAD_BLOCK, group_offsets=off)
+        mq.grouped_linear(Xq, Xsf, off, Wq, Wsf)
+    torch.cuda.synchronize(dev)
+    assert mq.device_status() == 0
+
+
 def profile_mode(M, steps, warmup, dev, form="layer"):
     """Eager layer passes with no timing: the commands the ncu captures run. form: "layer" (act_quant
-    then the GEMM), "fused" (the one-call layer from bf16 X), "w4a16" (the weight-only layer)."""
+    then the GEMM), "fused" (the one-call layer from bf16 X), "w4a16" (the weight-only layer), "moe"
+    (the MoE gate/up projection at T = 8192)."""
     import w4a4_mxfp4_quantized_b200 as mq
 
+    if form == "moe":
+        profile_moe(steps, warmup, dev)
+        return
     L = make_layer(M, dev, 2)
     for i in range(warmup + steps):
         if form == "fused":
